@@ -8,7 +8,10 @@ it imports nothing from the GPU library.
 discuss (PyTorch PR #126348's linear + cross-entropy steps, with the softmax
 rebuilt in backward from the logits and the per-row log-sum-exp; torchtune
 issue #1228's mean NLL against labels; Liger-Kernel issue #227's Gemma2 logit
-softcap).  The arithmetic lives in ``flce_oracle.c``; this module only
+softcap).  ``ce`` computes the same loss and its gradient with respect to
+the logits for a caller that already holds them (PR #126348's own case: the
+row max and sum in the forward, the softmax rebuilt from the logits in the
+backward).  The arithmetic lives in ``flce_oracle.c``; this module only
 marshals numpy arrays to it.
 """
 import ctypes
@@ -42,6 +45,9 @@ def _lib():
         lib.flce_oracle_count_valid.argtypes = [p, i64, i64]
         lib.flce_oracle_threads.restype = ctypes.c_int
         lib.flce_oracle_threads.argtypes = []
+        lib.flce_oracle_ce.restype = ctypes.c_int
+        lib.flce_oracle_ce.argtypes = [i64, i64, ctypes.c_int, p, i64, p, i64, ctypes.c_double,
+                                       i64, ctypes.c_double, p, p, p, p, p]
         _LIB = lib
     return _LIB
 
@@ -118,4 +124,43 @@ def flce(X, W, labels, ignore_index=-100, softcap=0.0, dloss=1.0, n_valid=None, 
     return out
 
 
-__all__ = ["flce", "count_valid", "threads", "OracleLabelError"]
+def ce(Z, labels, ignore_index=-100, softcap=0.0, dloss=1.0, n_valid=None, grads=True,
+       dtype=None, V=None):
+    """Cross-entropy in fp64 from logits the caller already holds (PyTorch
+    PR #126348's case: row max and sum in the forward, the softmax rebuilt
+    from the logits and the row statistics in the backward).
+
+    Z: [BT, ld] (float32 / float64, or raw bf16 bits with dtype="bf16"); the
+    logits of row i are Z[i, :V] (V defaults to ld, so extra columns model a
+    row stride).  labels: int64 [BT].  Returns a dict with lse, target,
+    n_valid, loss and, if grads, dZ [BT, V].
+    """
+    Za, code = _as_input(Z, dtype)
+    if Za.ndim != 2:
+        raise ValueError("Z must be [BT, ld]")
+    BT, ld = Za.shape
+    V = ld if V is None else int(V)
+    lab = np.ascontiguousarray(labels, dtype=np.int64)
+    if lab.shape != (BT,):
+        raise ValueError("labels must be [BT]")
+    lse = np.empty(BT, np.float64)
+    target = np.empty(BT, np.float64)
+    nv = ctypes.c_int64(0)
+    loss = ctypes.c_double(0.0)
+    dZ = np.empty((BT, V), np.float64) if grads else None
+    rc = _lib().flce_oracle_ce(
+        BT, V, code, Za.ctypes.data if BT else None, ld, lab.ctypes.data if BT else None,
+        int(ignore_index), float(softcap), -1 if n_valid is None else int(n_valid),
+        float(dloss), lse.ctypes.data, target.ctypes.data, ctypes.addressof(nv),
+        ctypes.addressof(loss), dZ.ctypes.data if grads else None)
+    if rc == 2:
+        raise OracleLabelError(_ERRORS[2])
+    if rc != 0:
+        raise RuntimeError("oracle failed: %s" % _ERRORS.get(rc, rc))
+    out = {"lse": lse, "target": target, "n_valid": int(nv.value), "loss": float(loss.value)}
+    if grads:
+        out["dZ"] = dZ
+    return out
+
+
+__all__ = ["flce", "ce", "count_valid", "threads", "OracleLabelError"]

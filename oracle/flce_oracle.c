@@ -230,3 +230,97 @@ int flce_oracle(int64_t BT, int64_t H, int64_t V, int dtype, const void* X, cons
   free(Z);
   return OR_OK;
 }
+
+/*
+ * Cross-entropy for a caller that already holds the logits ("softmax_input"),
+ * the exact case of PyTorch PR #126348 ("[AOTAutograd] tweak min-cut
+ * partitioner to avoid saving softmax output", summary steps 1-4 and points
+ * a./b.): the forward needs only the per-row max and sum (steps 2-3) and the
+ * label's entry (point a.); the backward rebuilds the softmax from the
+ * logits and those row statistics (point b.) instead of reading a saved
+ * softmax_output.  In fp64, with the same softcap, ignore_index and mean
+ * conventions as flce_oracle:
+ *
+ *   y_ij    = c*tanh(z_ij/c) under a softcap c, else z_ij
+ *   lse_i   = m_i + log sum_j exp(y_ij - m_i),  m_i = max_j y_ij
+ *   loss    = (1/N) sum_{valid i} (lse_i - y_{i,label_i}),  0 when N == 0
+ *   dZ_ij   = valid_i (exp(y_ij - lse_i) - [j == label_i]) s_ij dloss / N
+ *
+ * logits: BT rows of V entries, row i starting at element i*ld (ld >= V), in
+ * `dtype` (bf16 bits, fp32 or fp64).  n_valid < 0 counts N from these labels.
+ * Outputs: lse[BT], target[BT] (NaN on ignored rows), *n_valid_out,
+ * *loss_out and, when non-NULL, dZ (BT x V, dense, fp64).
+ */
+static double widen_at(const void* base, int dtype, int64_t idx) {
+  if (dtype == OR_BF16) return bf16_bits_to_double(((const uint16_t*)base)[idx]);
+  if (dtype == OR_FP32) return (double)((const float*)base)[idx];
+  return ((const double*)base)[idx];
+}
+
+int flce_oracle_ce(int64_t BT, int64_t V, int dtype, const void* logits, int64_t ld,
+                   const int64_t* labels, int64_t ignore_index, double softcap, int64_t n_valid,
+                   double dloss, double* lse, double* target, int64_t* n_valid_out,
+                   double* loss_out, double* dZ) {
+  int64_t i;
+  const int capped = softcap_on(softcap);
+  double loss = 0.0, scale;
+
+  if (BT < 0 || V <= 0 || ld < V || (dtype != OR_BF16 && dtype != OR_FP32 && dtype != OR_FP64))
+    return OR_INVALID;
+  if (BT > 0 && (!logits || !labels)) return OR_INVALID;
+  if (!lse || !target || !n_valid_out || !loss_out) return OR_INVALID;
+  for (i = 0; i < BT; ++i)
+    if (labels[i] != ignore_index && (labels[i] < 0 || labels[i] >= V)) return OR_BAD_LABEL;
+  if (n_valid < 0) n_valid = flce_oracle_count_valid(labels, BT, ignore_index);
+  *n_valid_out = n_valid;
+
+  /* Steps 2-3 per row: softcap, max, log-sum-exp; the label's entry. */
+#pragma omp parallel for schedule(static)
+  for (i = 0; i < BT; ++i) {
+    int64_t j;
+    double m = -INFINITY, s = 0.0;
+    for (j = 0; j < V; ++j) {
+      double z = widen_at(logits, dtype, i * ld + j);
+      double y = capped ? softcap * tanh(z / softcap) : z;
+      if (y > m) m = y;
+    }
+    for (j = 0; j < V; ++j) {
+      double z = widen_at(logits, dtype, i * ld + j);
+      double y = capped ? softcap * tanh(z / softcap) : z;
+      s += exp(y - m);
+    }
+    lse[i] = m + log(s);
+    if (labels[i] != ignore_index) {
+      double zt = widen_at(logits, dtype, i * ld + labels[i]);
+      target[i] = capped ? softcap * tanh(zt / softcap) : zt;
+    } else {
+      target[i] = NAN;
+    }
+  }
+
+  /* Mean NLL over the valid rows, summed in row order. */
+  for (i = 0; i < BT; ++i)
+    if (labels[i] != ignore_index) loss += lse[i] - target[i];
+  *loss_out = n_valid > 0 ? loss / (double)n_valid : 0.0;
+  if (!dZ) return OR_OK;
+
+  /* Backward: the softmax rebuilt from the logits and lse (point b.). */
+  scale = n_valid > 0 ? dloss / (double)n_valid : 0.0;
+#pragma omp parallel for schedule(static)
+  for (i = 0; i < BT; ++i) {
+    int64_t j;
+    const int valid = labels[i] != ignore_index;
+    for (j = 0; j < V; ++j) {
+      double g = 0.0;
+      if (valid && n_valid > 0) {
+        double z = widen_at(logits, dtype, i * ld + j);
+        double t = capped ? tanh(z / softcap) : 0.0;
+        double y = capped ? softcap * t : z;
+        double d = capped ? 1.0 - t * t : 1.0;
+        g = (exp(y - lse[i]) - (j == labels[i] ? 1.0 : 0.0)) * d * scale;
+      }
+      dZ[i * V + j] = g;
+    }
+  }
+  return OR_OK;
+}
