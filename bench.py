@@ -16,6 +16,15 @@ all-reduces the loss shares and dW (bf16) over NCCL.  --parallel replicas
 runs independent copies instead (no collective).  Time is the max over ranks
 of the device-timed region; value = tokens of all ranks / that time.
 
+--workload ce_llmc times the cross-entropy path for callers that already
+hold the logits (flce_ce_forward + flce_ce_backward) on PyTorch PR #126348's
+llm.c tensor (32 x 1024 rows, V = 50257, bf16): HBM-bound, one read of the
+logits forward, one read and one write backward.
+
+The headline loop is timed with two CUDA events and nothing else; per-kernel
+times (for the roofline and the shares) come from a second, shorter loop
+with an event pair around every launch.
+
 --impl reference times the fp64 CPU oracle (the only reference this build
 has) on a bounded row sample of the same workload, on rank 0 only.
 """
@@ -37,16 +46,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = ("FLCE fwd+bwd tokens/s and TFLOP/s (% of B200 BF16 peak); peak extra HBM GB")
 
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of each
-# kernel kind, from one full-size ncu capture of the Llama-3 workload with the
-# automatic schedule (profiles/launches_llama3_8b_fused.md; averages over the
-# two row chunks).  They describe the kernel code whose hash (csrc_sha16) is
-# recorded here and are reported as null for any other build.
-TRAFFIC = {
-    "csrc_sha16": "dd26121eadcb90f6", "workload": "llama3_8b", "schedule": "auto",
-    "bytes_per_launch": {"lse_p_gemm": 3.420e9, "dx_gemm": 8.997e9, "dw_acc_gemm": 5.922e9,
-                         "lse_grad": 2.011e9},
-}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per launch of a
+# kernel kind, from single-kernel ncu captures of the named workload (the
+# commands and the per-launch figures are kept under profiles/).  They
+# describe the kernel code whose hash (csrc_sha16) is recorded with them and
+# are reported as null for any other build or workload.
+TRAFFIC = {}
 
 
 def csrc_sha16(root=None):
@@ -204,22 +209,31 @@ def run_reference(args, world, rank):
     if rank != 0:
         return
     from linear_cross_entropy_tiles_b200 import inputs
-    w = inputs.WORKLOADS[args.workload]
-    X, W, labels = inputs.make_workload(w, device="cuda")
-    rows = args.cpu_rows
+    if args.workload.startswith("ce_"):
+        w = inputs.CE_WORKLOADS[args.workload]
+        Z, labels = inputs.make_ce_workload(w, device="cuda")
+        rows = args.ce_cpu_rows
+        sample, metric, config = (lambda: ce_oracle_sample(w, Z, labels, rows), CE_METRIC,
+                                  ce_config(w, world))
+    else:
+        w = inputs.WORKLOADS[args.workload]
+        X, W, labels = inputs.make_workload(w, device="cuda")
+        rows = args.cpu_rows
+        sample, metric, config = (lambda: cpu_oracle_sample(w, X, W, labels, rows), METRIC,
+                                  workload_config(w, world))
     times = []
     cb = None
     for i in range(args.warmup + args.steps):
-        cb = cpu_oracle_sample(w, X, W, labels, rows)
+        cb = sample()
         if i >= args.warmup:
             times.append(rows / cb["value"])
     t = sum(times) / len(times)
     value = rows / t
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+    line = {"impl": "reference", "metric": metric, "value": value, "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, world),
+            "config": config,
             "cpu_baseline": dict(cb, value=value),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -227,13 +241,50 @@ def run_reference(args, world, rank):
 
 
 def traffic_of(kind, workload, schedule, bt_override):
-    """DRAM bytes per launch of `kind` from the recorded capture, or None when
-    the capture does not describe this build and workload."""
-    t = TRAFFIC
-    if (bt_override or workload != t["workload"] or schedule != t["schedule"]
-            or csrc_sha16() != t["csrc_sha16"]):
+    """DRAM bytes per launch of `kind` from the recorded captures, or None when
+    no capture describes this build, workload and schedule."""
+    t = TRAFFIC.get((workload, schedule))
+    if bt_override or t is None or csrc_sha16() != t["csrc_sha16"]:
         return None
     return t["bytes_per_launch"].get(kind)
+
+
+def profile_kinds(step, n_steps, launches_per_step):
+    """Run n_steps of `step` with an event pair around every library launch;
+    return {kind: [total ms, launches]}."""
+    import linear_cross_entropy_tiles_b200 as flce
+    torch.cuda.synchronize()
+    flce.flce_profile_start(launches_per_step * n_steps + 8)
+    for _ in range(n_steps):
+        step()
+    torch.cuda.synchronize()
+    by_kind = {}
+    for name, t in flce.flce_profile_stop():
+        k = by_kind.setdefault(name, [0.0, 0])
+        k[0] += t
+        k[1] += 1
+    return by_kind
+
+
+def time_steps(step, steps, world, stream, sampler=None):
+    """Device time of `steps` calls of step() between two CUDA events on the
+    launching stream, barriers and synchronisation on both sides; ms per
+    step, max over ranks."""
+    barrier(world)
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.start()
+        time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop() if sampler is not None else None
+    return max_over_ranks(t0.elapsed_time(t1) / steps, world), clocks
 
 
 def workload_config(w, world, parallel="replicas"):
@@ -314,6 +365,127 @@ def run_ragged(args, world, rank):
             "gpu_launches": launches, "clocks": clocks, "per_bt": per_bt}), flush=True)
 
 
+CE_METRIC = ("cross-entropy from held logits, fwd+bwd tokens/s and GB/s (% of B200 HBM "
+             "copy bandwidth)")
+
+
+def ce_config(w, world):
+    return {"workload": "%s: logits BT=%d x V=%d %s (PyTorch PR #126348's llm.c tensor), "
+                        "N(0, %.3f^2), %.0f%% ignored" % (w.name, w.BT, w.V, w.dtype, w.std,
+                                                         100 * w.ignore_frac),
+            "BT": w.BT, "V": w.V, "softcap": w.softcap, "seed": w.seed,
+            "l2": "inputs larger than L2 (logits %.2f GB vs 126 MB L2)"
+                  % (w.BT * w.V * 2 / 1e9),
+            "parallelism": "replicas x%d" % world}
+
+
+def ce_oracle_sample(w, Z, labels, rows):
+    """Time the fp64 oracle's cross-entropy (forward and gradient) on `rows`
+    rows of the logits."""
+    import oracle
+    from linear_cross_entropy_tiles_b200 import inputs
+    R = inputs.sample_rows(w.BT, rows, seed=7)
+    za, tag = inputs.oracle_view(Z[R].cpu())
+    lab = labels[R].cpu().numpy()
+    nv = int((labels != inputs.IGNORE_INDEX).sum().item())
+    t0 = time.perf_counter()
+    oracle.ce(za, lab, softcap=w.softcap, n_valid=nv, dtype=tag)
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": "tokens/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": "%d of %d rows (full V=%d), fp64 forward + logit gradient; %.2f s"
+                      % (rows, w.BT, w.V, dt)}
+
+
+def run_ce(args, world, rank):
+    """flce_ce_forward + flce_ce_backward on logits resident in HBM."""
+    import linear_cross_entropy_tiles_b200 as flce
+    from linear_cross_entropy_tiles_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = inputs.CE_WORKLOADS[args.workload]
+    if args.bt:
+        import dataclasses
+        w = dataclasses.replace(w, BT=args.bt)
+    Z, labels = inputs.make_ce_workload(w, device=dev)
+    stream = torch.cuda.current_stream()
+    pf = flce.make_ce_problem(w.BT, w.V, Z.dtype, softcap=w.softcap)
+    ws_f = flce.ce_workspace(pf, flce.FLCE_OP_FORWARD, dev)
+    ws_b = flce.ce_workspace(pf, flce.FLCE_OP_BACKWARD, dev)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    lse = torch.empty(w.BT, dtype=torch.float32, device=dev)
+    dloss = torch.ones(1, dtype=torch.float32, device=dev)
+    dZ = torch.empty_like(Z)
+
+    def step():
+        flce.flce_ce_forward(pf, Z, labels, loss, lse, ws_f, stream)
+        flce.flce_ce_backward(pf, Z, labels, lse, dloss, dZ, ws_b, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status, n_valid = flce.flce_get_device_status(ws_f)
+    if status != 0:
+        raise SystemExit("device status %d after warm-up" % status)
+    flce.flce_ce_forward(pf, Z, labels, loss, lse, ws_f, stream)
+    launches_per_step = flce.flce_last_launch_count()
+    flce.flce_ce_backward(pf, Z, labels, lse, dloss, dZ, ws_b, stream)
+    launches_per_step += flce.flce_last_launch_count()
+    sampler = ClockSampler(torch.cuda.current_device())
+    ms, clocks = time_steps(step, args.steps, world, stream, sampler)
+    peaks = load_peaks()
+    by_kind = profile_kinds(step, max(1, min(args.steps, args.prof_steps)), launches_per_step)
+    total = sum(v[0] for v in by_kind.values())
+    elem = w.BT * w.V * (2 if w.dtype == "bf16" else 4)
+    # The backward moves two of the step's three logits-sized passes.
+    bytes_per_launch = {"ce_forward": float(elem), "ce_backward": 2.0 * elem}
+    dom = max(by_kind, key=lambda n: by_kind[n][0])
+    dom_ms = by_kind[dom][0] / by_kind[dom][1]
+    achieved = bytes_per_launch.get(dom, 0.0) / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "peak_kind": "%s HBM copy bandwidth" % peaks["source"],
+                "bytes_per_launch": bytes_per_launch.get(dom), "avg_launch_ms": dom_ms,
+                "traffic": traffic_of(dom, args.workload, "auto", args.bt),
+                "per_kernel_gbs": {k: round(bytes_per_launch[k] / (v[0] / v[1] / 1e3) / 1e9, 1)
+                                   for k, v in by_kind.items() if k in bytes_per_launch},
+                "shares": {k: round(v[0] / total, 4) for k, v in sorted(by_kind.items())}}
+    e2e = None
+    if not args.no_e2e:
+        Zh = Z.cpu().pin_memory()
+        Lh = labels.cpu().pin_memory()
+        lossh = torch.empty(1, dtype=torch.float32).pin_memory()
+        dZh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
+
+        def e2e_step():
+            Z.copy_(Zh, non_blocking=True)
+            labels.copy_(Lh, non_blocking=True)
+            step()
+            lossh.copy_(loss, non_blocking=True)
+            dZh.copy_(dZ, non_blocking=True)
+
+        e2e_step()
+        ems, _ = time_steps(e2e_step, args.e2e_steps, world, stream)
+        e2e = {"value": world * w.BT / (ems / 1e3), "unit": "tokens/s", "ms_per_step": ems,
+               "h2d_bytes_per_step": Zh.numel() * Zh.element_size() + Lh.numel() * 8,
+               "d2h_bytes_per_step": 4 + dZh.numel() * dZh.element_size(),
+               "api": "linear_cross_entropy_tiles_b200 flce_ce_forward + flce_ce_backward "
+                      "(C ABI)"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = ce_oracle_sample(w, Z, labels, args.ce_cpu_rows)
+    if rank == 0:
+        print(json.dumps({
+            "metric": CE_METRIC, "value": world * w.BT / (ms / 1e3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic", "config": ce_config(w, world),
+            "gbs": w.bytes_per_step / (ms / 1e3) / 1e9,
+            "frac_of_hbm": w.bytes_per_step / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "bytes_per_step": w.bytes_per_step, "n_valid": n_valid,
+            "loss": float(loss.item()), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps, "clocks": clocks}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -326,11 +498,14 @@ def main():
     ap.add_argument("--schedule", default="auto", choices=["auto", "recompute", "fused_fwd"],
                     help="flce_fused schedule (auto: fused-in-forward for BT >= 512)")
     ap.add_argument("--cpu-rows", type=int, default=8)
+    ap.add_argument("--ce-cpu-rows", type=int, default=8192)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ragged-reps", type=int, default=3)
     ap.add_argument("--ragged-limit", type=int, default=0)
+    ap.add_argument("--prof-steps", type=int, default=20,
+                    help="steps of the second, per-launch-timed loop")
     ap.add_argument("--parallel", default=None, choices=["dp", "replicas"],
                     help="with several ranks: data parallel over rows (default) or "
                          "independent replicas; 'dp' on one rank runs the same step "
@@ -339,8 +514,9 @@ def main():
     world_env = int(os.environ.get("WORLD_SIZE", "1"))
     if args.parallel is None:
         args.parallel = "dp" if world_env > 1 else "replicas"
-    if args.workload == "ragged" and args.parallel == "dp":
-        args.parallel = "replicas"  # the ragged sweep runs each BT as its own problem
+    if (args.workload == "ragged" or args.workload.startswith("ce_")) and args.parallel == "dp":
+        # each ragged BT is a problem of its own; the CE path has no exchange
+        args.parallel = "replicas"
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
@@ -353,6 +529,11 @@ def main():
 
     if args.workload == "ragged":
         run_ragged(args, world, rank)
+        finish(world)
+        return
+
+    if args.workload.startswith("ce_"):
+        run_ce(args, world, rank)
         finish(world)
         return
 
@@ -408,33 +589,14 @@ def main():
     extra_bytes = ws.numel()  # the only scratch memory; the library allocates nothing
 
     sampler = ClockSampler(torch.cuda.current_device())
-    flce.flce_profile_start(launches_per_step * args.steps + 8)
-    barrier(world)
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.3)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        step()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks = sampler.stop()
-    prof = flce.flce_profile_stop()
-    ms_local = t0.elapsed_time(t1) / args.steps
-    ms = max_over_ranks(ms_local, world)
+    ms, clocks = time_steps(step, args.steps, world, stream, sampler)
     tokens_per_s = world * w.BT / (ms / 1e3)
     tflops = world * w.flops / (ms / 1e3) / 1e12
     peaks = load_peaks()
 
-    # Dominant kernel: the GEMM kind with the largest share of device time.
-    by_kind = {}
-    for name, t in prof:
-        k = by_kind.setdefault(name, [0.0, 0])
-        k[0] += t
-        k[1] += 1
+    # Per-kernel times from a second loop with events around every launch.
+    prof_steps = max(1, min(args.steps, args.prof_steps))
+    by_kind = profile_kinds(step, prof_steps, launches_per_step)
     total_prof = sum(v[0] for v in by_kind.values())
     dom = max(by_kind, key=lambda n: by_kind[n][0])
     # Algorithmic FLOPs per step of each GEMM kind: 2*BT*H*V each (the LSE and
@@ -443,12 +605,15 @@ def main():
     flops_per_step = {k: gemm_flops for k in ("lse_gemm", "grad_gemm", "dx_gemm", "dw_gemm",
                                               "lse_p_gemm", "dw_acc_gemm", "simt_lse",
                                               "simt_grad", "simt_dx", "simt_dw")}
-    dom_time_per_step = by_kind[dom][0] / args.steps
-    launches_dom = by_kind[dom][1] / args.steps
+    dom_time_per_step = by_kind[dom][0] / prof_steps
+    launches_dom = by_kind[dom][1] / prof_steps
     achieved = flops_per_step.get(dom, 0.0) / (dom_time_per_step / 1e3) / 1e12
     if w.dtype == "bf16":
-        bound, peak = "tensor", peaks["bf16_sustained"]
-        peak_kind = "%s sustained dense bf16 (cuBLAS loop)" % peaks["source"]
+        # A kernel of a few ms timed inside a sub-second region: the burst peak.
+        bound, peak = "tensor", peaks["bf16"]
+        peak_kind = ("%s burst dense bf16 (cuBLAS GEMM timed alone); frac_sustained divides "
+                     "by the %s sustained figure (cuBLAS loop under the power cap)"
+                     % (peaks["source"], peaks["source"]))
     else:
         # fp32 FMA on CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
         bound, peak = "alu", 148 * 128 * 2 * 1.965e9 / 1e12
@@ -456,7 +621,9 @@ def main():
     roofline = {"bound": bound, "kernel": dom, "achieved": achieved,
                 "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak,
-                "peak_kind": peak_kind,
+                "frac_sustained": (achieved / peaks["bf16_sustained"]
+                                   if w.dtype == "bf16" else None),
+                "peak_kind": peak_kind, "profiled_steps": prof_steps,
                 "flops_per_launch": flops_per_step.get(dom, 0.0) / launches_dom,
                 "avg_launch_ms": dom_time_per_step / launches_dom,
                 "traffic": traffic_of(dom, args.workload, args.schedule, args.bt),

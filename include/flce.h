@@ -28,9 +28,15 @@
  *
  * Conventions for every entry point:
  *   - All array arguments are DEVICE pointers (memory the caller allocated on
- *     the current CUDA device), row-major and dense: X is BT x H with row
- *     stride H, W is V x H with row stride H, dX like X, dW like W.
- *     X, W, dX and dW must be 16-byte aligned; labels 8-byte aligned.
+ *     the current CUDA device), row-major: X is BT x H with row stride ldx
+ *     elements, W is V x H with row stride ldw, dX is BT x H with row stride
+ *     lddx, dW is V x H with row stride lddw (each 0 = H, dense).  A stride
+ *     lets X be a slice of a wider activation (hidden[:, a:a+H]), W a slice
+ *     of a padded or tied weight, and the gradients land inside wider
+ *     buffers, with no copy.  Every row must start on a 16-byte boundary:
+ *     X, W, dX and dW 16-byte aligned and each stride times the element size
+ *     a multiple of 16 (else FLCE_ERR_MISALIGNED); a stride below H is
+ *     FLCE_ERR_INVALID_ARG.  labels is dense, 8-byte aligned.
  *     labels is int64 [BT]: per-row labels, or token ids that the op shifts
  *     itself when flce_problem_t.shift_seq_len > 0.
  *   - Element type: FLCE_BF16 (bfloat16 X/W/dX/dW, fp32 accumulation, the
@@ -86,7 +92,7 @@ typedef enum { FLCE_BF16 = 0, FLCE_FP32 = 1 } flce_dtype_t;
 typedef enum { FLCE_OP_FORWARD = 0, FLCE_OP_BACKWARD = 1, FLCE_OP_FUSED = 2 } flce_op_t;
 
 /* Problem description.  softcap <= 0, NaN or +inf means "no softcap".
- * Size limits (else FLCE_ERR_UNSUPPORTED): BT, H, V < 2^31;
+ * Size limits (else FLCE_ERR_UNSUPPORTED): BT, H, V < 2^31; strides < 2^31;
  * ceil(BT/128) * ceil(V/256) < 2^28 (32-bit tile ids); fp32 problems
  * BT <= 65535 * 32. */
 typedef struct {
@@ -100,7 +106,16 @@ typedef struct {
                            position is ignored); BT must be a multiple of T */
   int64_t ignore_index; /* label value that marks a row as ignored (e.g. -100) */
   float softcap;        /* Gemma2-style logit cap c, or <= 0 for none */
-  int32_t reserved1;    /* must be 0 */
+  int32_t dw_fp32;      /* 0: dW has X's element type; 1: dW is fp32 (V x H
+                           float, row stride lddw) whatever X's type, for a
+                           gradient kept, or summed over ranks, in fp32.  With
+                           bf16 inputs the fused-in-forward schedule then keeps
+                           its running sum of dW in dW itself instead of the
+                           workspace.  Other values: FLCE_ERR_INVALID_ARG */
+  int64_t ldx;          /* row stride of X in elements; 0 = H */
+  int64_t ldw;          /* row stride of W in elements; 0 = H */
+  int64_t lddx;         /* row stride of dX in elements; 0 = H */
+  int64_t lddw;         /* row stride of dW in elements; 0 = H */
 } flce_problem_t;
 
 /* Bytes of workspace `op` (flce_op_t) needs for problem `p`, or 0 when `p`
@@ -174,9 +189,11 @@ FLCE_API flce_status_t flce_fused_global(const flce_problem_t* p, const void* X,
  * GPU which loads it keeps until the process exits; the call allocates
  * nothing.  Problems whose fused workspace (flce_workspace_size(p,
  * FLCE_OP_FUSED)) is larger are rejected with FLCE_ERR_WORKSPACE_TOO_SMALL
- * before any work is enqueued.  The first call on each device looks up the
- * array's device address on that device (make that first call before any
- * stream capture).  All calls on a device share the one array and it keeps
+ * before any work is enqueued.  Every call looks up the array's address in
+ * the current device's context; the first call on a device may load the
+ * library's device code to do so, so it must not be made while `stream` is
+ * being captured into a CUDA graph (it then returns FLCE_ERR_INVALID_ARG
+ * without enqueueing anything).  All calls on a device share the one array and it keeps
  * the previous call's contents; the computation overwrites every scratch
  * byte before reading it, so nothing needs clearing, but calls whose GPU
  * work overlaps race on the array: serialise them.  The device status of a
@@ -185,6 +202,66 @@ FLCE_API flce_status_t flce_fused_global(const flce_problem_t* p, const void* X,
 FLCE_API flce_status_t flce_fused_noalloc(const flce_problem_t* p, const void* X, const void* W,
                                           const int64_t* labels, float dloss, float* loss,
                                           void* dX, void* dW, struct CUstream_st* stream);
+
+/* ---------------- cross-entropy for callers that hold the logits -------------
+ *
+ * PyTorch PR #126348's own case: the caller already has softmax_input (the
+ * logits, BT x V), e.g. from its own LM-head matmul.  The PR's summary lists
+ * the unfused loss as a matmul then three passes over the logits (row max,
+ * row sum, a normalised softmax_output saved for backward) and observes that
+ * (a.) the forward needs only the label's entry of the softmax and (b.) the
+ * backward can rebuild the softmax from the logits and the small row
+ * statistics.  flce_ce_forward reads the logits once and keeps only
+ * lse [BT]; flce_ce_backward reads them once more and writes the gradient,
+ * rebuilding the softmax from the logits and that lse.  Nothing else of size
+ * BT x V is read or written.
+ *
+ *   y     = c tanh(z / c) under a softcap c, else z       (z: the logits)
+ *   lse_i = log sum_j exp(y_ij)
+ *   loss  = mean over rows with label_i != ignore_index of (lse_i - y_i,label_i)
+ *   dZ_ij = (exp(y_ij - lse_i) - [j == label_i]) * dy/dz * dloss / N_valid,
+ *           rows with ignored labels zero
+ *
+ * Same conventions as the FLCE calls above (labels, shift_seq_len,
+ * ignore_index, softcap, the all-ignored case, device status word, stream,
+ * caller-owned workspace), except the layout:
+ *   - logits and dlogits are DEVICE arrays of BT rows of V entries (bf16 or
+ *     fp32, `dtype`), row i at element i*ld (resp. i*ld_grad); ld = 0 means
+ *     V.  Rows need not be 16-byte aligned (a dense bf16 tensor with odd V is
+ *     fine); the pointers must be aligned to the element size.
+ *   - dlogits may be the logits array itself (ld_grad == ld): the gradient
+ *     then overwrites the logits in place.  Any other overlap is undefined.
+ * Size limits: BT, V < 2^31; ld, ld_grad < 2^40 (else FLCE_ERR_UNSUPPORTED);
+ * ld or ld_grad below V is FLCE_ERR_INVALID_ARG. */
+typedef struct {
+  int64_t BT;            /* rows, >= 0 */
+  int64_t V;             /* classes (vocabulary), > 0 */
+  int32_t dtype;         /* flce_dtype_t of logits and dlogits */
+  int32_t shift_seq_len; /* as in flce_problem_t */
+  int64_t ignore_index;
+  float softcap;         /* <= 0, NaN or inf: none */
+  int32_t reserved1;     /* must be 0 */
+  int64_t ld;            /* row stride of logits in elements; 0 = V */
+  int64_t ld_grad;       /* row stride of dlogits in elements; 0 = V */
+} flce_ce_problem_t;
+
+/* Workspace bytes for op FLCE_OP_FORWARD or FLCE_OP_BACKWARD (0 when the
+ * problem or op is invalid): a 256-byte header, [BT] fp32 per-row losses
+ * (forward), [BT] int64 shifted labels (shift_seq_len > 0). */
+FLCE_API size_t flce_ce_workspace_size(const flce_ce_problem_t* p, int op);
+
+/* loss (device fp32 scalar) and lse (device fp32 [BT], kept for
+ * flce_ce_backward) from the logits: one read of them. */
+FLCE_API flce_status_t flce_ce_forward(const flce_ce_problem_t* p, const void* logits,
+                                       const int64_t* labels, float* loss, float* lse, void* ws,
+                                       size_t ws_bytes, struct CUstream_st* stream);
+
+/* dlogits from the logits, the forward's lse and the upstream gradient dloss
+ * (device fp32 scalar): one read of the logits, one write of dlogits. */
+FLCE_API flce_status_t flce_ce_backward(const flce_ce_problem_t* p, const void* logits,
+                                        const int64_t* labels, const float* lse,
+                                        const float* dloss, void* dlogits, void* ws,
+                                        size_t ws_bytes, struct CUstream_st* stream);
 
 /* How flce_fused schedules its work (bf16 problems; fp32 always recomputes).
  *  FLCE_SCHEDULE_RECOMPUTE: forward pass for lse and loss, then per
@@ -205,6 +282,17 @@ typedef enum {
  * flce_workspace_size for FLCE_OP_FUSED); returns the previous one, or -1
  * for an unknown value. */
 FLCE_API int32_t flce_set_schedule(int32_t schedule);
+
+/* Process-wide cap, in bytes, on the workspace flce_fused plans under
+ * FLCE_SCHEDULE_AUTO (0 = none, the default; also used by
+ * flce_workspace_size for FLCE_OP_FUSED).  Under the cap AUTO takes the
+ * fused-in-forward schedule only when its workspace fits, else the
+ * recompute schedule with its vocabulary chunk narrowed (down to 256
+ * columns) until the workspace fits; when nothing fits it plans the
+ * smallest recompute workspace.  A cap of one bf16 BT x V tensor (2*BT*V
+ * bytes) keeps every plan below the logits' size.  The forced schedules
+ * ignore it.  Returns the previous cap. */
+FLCE_API uint64_t flce_set_workspace_limit(uint64_t bytes);
 
 /* Synchronise `stream`, then read the device status word and the valid-row
  * count of the last call that used workspace `ws`.  Either output pointer
@@ -232,6 +320,15 @@ FLCE_API int32_t flce_last_launch_count(void);
  * first).  Read it with flce_get_device_status; the context stays usable. */
 FLCE_API flce_status_t flce_selftest_wait_timeout(void* ws, uint64_t limit_ns,
                                                   struct CUstream_st* stream);
+
+/* Accuracy self-test of the two approximations the GEMM epilogues use in
+ * place of library calls: for each of the n fp32 inputs x[i] (device),
+ * out[4i .. 4i+3] (device fp32) = the epilogues' tanh (1 - 2 / (2^(2x log2 e)
+ * + 1) on the hardware exp2), CUDA's tanhf, the epilogues' exp2 (the
+ * ex2.approx.ftz instruction) and CUDA's exp2f, so a test can bound the
+ * difference.  Enqueued on `stream`. */
+FLCE_API flce_status_t flce_selftest_approx(const float* x, int64_t n, float* out,
+                                            struct CUstream_st* stream);
 
 /* Per-launch timing for profiling.  flce_profile_start(n) creates 2n CUDA
  * events; until flce_profile_stop, every kernel the library launches records

@@ -1,8 +1,12 @@
 """ctypes binding of the FLCE C ABI (include/flce.h).
 
 The functions here carry the C names and only marshal arguments: torch
-tensors become device pointers, the problem becomes an ``flce_problem_t``,
-and a non-OK status becomes an ``FlceError``.  Every step of the computation
+tensors become device pointers, the problem becomes an ``flce_problem_t``
+(or ``flce_ce_problem_t``), and a non-OK status becomes an ``FlceError``.
+Before a pointer is taken, each tensor is checked against the problem it is
+passed with (shape, element type, row stride, device), and a mismatch
+raises ``ValueError``: the C ABI sees only addresses and sizes, so a tensor
+whose layout differs from the problem's would otherwise be read wrongly.  Every step of the computation
 runs in the CUDA kernels of ``_build/libflce.so``; if that library is missing
 the first call raises instead of computing anything another way.
 """
@@ -30,7 +34,9 @@ EXPORTS = ("flce_workspace_size", "flce_forward", "flce_backward", "flce_fused",
            "flce_get_device_status", "flce_status_string", "flce_set_wait_limit_ns",
            "flce_last_launch_count", "flce_profile_start", "flce_profile_stop",
            "flce_kernel_name", "flce_fused_noalloc", "flce_set_schedule",
-           "flce_selftest_wait_timeout", "flce_count_valid", "flce_fused_global")
+           "flce_selftest_wait_timeout", "flce_count_valid", "flce_fused_global",
+           "flce_ce_workspace_size", "flce_ce_forward", "flce_ce_backward",
+           "flce_selftest_approx", "flce_set_workspace_limit")
 FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_RECOMPUTE, FLCE_SCHEDULE_FUSED_FORWARD = 0, 1, 2
 
 
@@ -45,7 +51,15 @@ class flce_problem_t(ctypes.Structure):
     _fields_ = [("BT", ctypes.c_int64), ("H", ctypes.c_int64), ("V", ctypes.c_int64),
                 ("dtype", ctypes.c_int32), ("shift_seq_len", ctypes.c_int32),
                 ("ignore_index", ctypes.c_int64), ("softcap", ctypes.c_float),
-                ("reserved1", ctypes.c_int32)]
+                ("dw_fp32", ctypes.c_int32), ("ldx", ctypes.c_int64), ("ldw", ctypes.c_int64),
+                ("lddx", ctypes.c_int64), ("lddw", ctypes.c_int64)]
+
+
+class flce_ce_problem_t(ctypes.Structure):
+    _fields_ = [("BT", ctypes.c_int64), ("V", ctypes.c_int64), ("dtype", ctypes.c_int32),
+                ("shift_seq_len", ctypes.c_int32), ("ignore_index", ctypes.c_int64),
+                ("softcap", ctypes.c_float), ("reserved1", ctypes.c_int32),
+                ("ld", ctypes.c_int64), ("ld_grad", ctypes.c_int64)]
 
 
 _LIB = None
@@ -95,16 +109,42 @@ def lib():
         L.flce_fused_global.restype = ctypes.c_int
         L.flce_fused_global.argtypes = [P, p, p, p, p, ctypes.c_float, p, p, p, p,
                                         ctypes.c_size_t, p]
+        L.flce_set_workspace_limit.restype = ctypes.c_uint64
+        L.flce_set_workspace_limit.argtypes = [ctypes.c_uint64]
+        L.flce_selftest_approx.restype = ctypes.c_int
+        L.flce_selftest_approx.argtypes = [p, ctypes.c_int64, p, p]
+        C = ctypes.POINTER(flce_ce_problem_t)
+        L.flce_ce_workspace_size.restype = ctypes.c_size_t
+        L.flce_ce_workspace_size.argtypes = [C, ctypes.c_int]
+        L.flce_ce_forward.restype = ctypes.c_int
+        L.flce_ce_forward.argtypes = [C, p, p, p, p, p, ctypes.c_size_t, p]
+        L.flce_ce_backward.restype = ctypes.c_int
+        L.flce_ce_backward.argtypes = [C, p, p, p, p, p, p, ctypes.c_size_t, p]
         _LIB = L
     return _LIB
 
 
+_DTYPES = {torch.bfloat16: FLCE_BF16, torch.float32: FLCE_FP32}
+
+
+def _dtype_code(dtype):
+    return _DTYPES.get(dtype, 99) if isinstance(dtype, torch.dtype) else int(dtype)
+
+
 def make_problem(BT, H, V, dtype=FLCE_BF16, ignore_index=-100, softcap=0.0,
-                 shift_seq_len=0) -> flce_problem_t:
-    if isinstance(dtype, torch.dtype):
-        dtype = {torch.bfloat16: FLCE_BF16, torch.float32: FLCE_FP32}.get(dtype, 99)
-    return flce_problem_t(int(BT), int(H), int(V), int(dtype), int(shift_seq_len),
-                          int(ignore_index), float(softcap), 0)
+                 shift_seq_len=0, ldx=0, ldw=0, lddx=0, lddw=0, dw_fp32=0) -> flce_problem_t:
+    """An flce_problem_t; the row strides ld* are in elements, 0 = H;
+    dw_fp32 = 1 asks for an fp32 dW whatever the input type."""
+    return flce_problem_t(int(BT), int(H), int(V), _dtype_code(dtype), int(shift_seq_len),
+                          int(ignore_index), float(softcap), int(dw_fp32), int(ldx), int(ldw),
+                          int(lddx), int(lddw))
+
+
+def make_ce_problem(BT, V, dtype=FLCE_BF16, ignore_index=-100, softcap=0.0, shift_seq_len=0,
+                    ld=0, ld_grad=0) -> flce_ce_problem_t:
+    """An flce_ce_problem_t; ld, ld_grad are row strides in elements, 0 = V."""
+    return flce_ce_problem_t(int(BT), int(V), _dtype_code(dtype), int(shift_seq_len),
+                             int(ignore_index), float(softcap), 0, int(ld), int(ld_grad))
 
 
 def _ptr(t):
@@ -113,6 +153,77 @@ def _ptr(t):
     if isinstance(t, int):
         return t
     return t.data_ptr() if t.numel() > 0 else None
+
+
+def _row_stride(t):
+    """Elements between rows of a 2-D tensor whose rows are unit-stride."""
+    if t.dim() != 2:
+        raise ValueError("expected a 2-D tensor, got shape %s" % (tuple(t.shape),))
+    if t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError("rows must be unit-stride (got strides %s)" % (t.stride(),))
+    return t.stride(0) if t.shape[0] > 1 else t.shape[1]
+
+
+def _check_matrix(name, t, rows, cols, dtype_code, ld, device):
+    """Raise unless tensor t is a rows x cols matrix of the problem's dtype
+    whose rows lie ld elements apart (0 = cols), on `device`."""
+    if not isinstance(t, torch.Tensor):
+        return device  # a raw address: the caller vouches for it
+    if tuple(t.shape) != (rows, cols):
+        raise ValueError("%s: shape %s, the problem says (%d, %d)"
+                         % (name, tuple(t.shape), rows, cols))
+    if _DTYPES.get(t.dtype) != dtype_code:
+        raise ValueError("%s: dtype %s does not match the problem's" % (name, t.dtype))
+    if rows > 1 and cols > 0 and _row_stride(t) != (ld or cols):
+        raise ValueError("%s: row stride %d, the problem says %d"
+                         % (name, _row_stride(t), ld or cols))
+    if t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError("%s: rows must be unit-stride" % name)
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (got %s)" % (name, t.device))
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, other arguments on %s" % (name, t.device, device))
+    return t.device
+
+
+def _check_vector(name, t, n, dtype, device):
+    if not isinstance(t, torch.Tensor):
+        return device
+    if t.dtype != dtype or t.numel() != n or (n > 1 and not t.is_contiguous()):
+        raise ValueError("%s: need a dense %s tensor of %d elements, got %s %s"
+                         % (name, dtype, n, t.dtype, tuple(t.shape)))
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (got %s)" % (name, t.device))
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, other arguments on %s" % (name, t.device, device))
+    return t.device
+
+
+def _check_flce(p, X=None, W=None, labels=None, dX=None, dW=None, lse=None, extra=()):
+    """Tensors passed with an flce_problem_t must be laid out as it says."""
+    dev = None
+    dev = _check_matrix("X", X, p.BT, p.H, p.dtype, p.ldx, dev)
+    dev = _check_matrix("W", W, p.V, p.H, p.dtype, p.ldw, dev)
+    dev = _check_matrix("dX", dX, p.BT, p.H, p.dtype, p.lddx, dev)
+    dev = _check_matrix("dW", dW, p.V, p.H, FLCE_FP32 if p.dw_fp32 else p.dtype, p.lddw, dev)
+    dev = _check_vector("labels", labels, p.BT, torch.int64, dev)
+    dev = _check_vector("lse", lse, p.BT, torch.float32, dev)
+    for name, t, n, dt in extra:
+        dev = _check_vector(name, t, n, dt, dev)
+
+
+def _check_ce(p, logits=None, labels=None, lse=None, dlogits=None, extra=()):
+    dev = None
+    dev = _check_matrix("logits", logits, p.BT, p.V, p.dtype, p.ld, dev)
+    dev = _check_matrix("dlogits", dlogits, p.BT, p.V, p.dtype, p.ld_grad, dev)
+    dev = _check_vector("labels", labels, p.BT, torch.int64, dev)
+    dev = _check_vector("lse", lse, p.BT, torch.float32, dev)
+    for name, t, n, dt in extra:
+        dev = _check_vector(name, t, n, dt, dev)
+
+
+def _nbytes(ws):
+    return ws.numel() * ws.element_size()
 
 
 def _stream(stream):
@@ -135,18 +246,24 @@ def flce_workspace_size(problem: flce_problem_t, op: int) -> int:
 
 
 def flce_forward(problem, X, W, labels, loss, lse, ws, stream=None):
+    _check_flce(problem, X=X, W=W, labels=labels, lse=lse,
+                extra=[("loss", loss, 1, torch.float32)])
     _check(lib().flce_forward(ctypes.byref(problem), _ptr(X), _ptr(W), _ptr(labels), _ptr(loss),
                               _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
                               _stream(stream)), "flce_forward")
 
 
 def flce_backward(problem, X, W, labels, lse, dloss, dX, dW, ws, stream=None):
+    _check_flce(problem, X=X, W=W, labels=labels, lse=lse, dX=dX, dW=dW,
+                extra=[("dloss", dloss, 1, torch.float32)])
     _check(lib().flce_backward(ctypes.byref(problem), _ptr(X), _ptr(W), _ptr(labels), _ptr(lse),
                                _ptr(dloss), _ptr(dX), _ptr(dW), _ptr(ws),
                                ws.numel() * ws.element_size(), _stream(stream)), "flce_backward")
 
 
 def flce_fused(problem, X, W, labels, dloss, loss, dX, dW, ws, stream=None):
+    _check_flce(problem, X=X, W=W, labels=labels, dX=dX, dW=dW,
+                extra=[("loss", loss, 1, torch.float32)])
     _check(lib().flce_fused(ctypes.byref(problem), _ptr(X), _ptr(W), _ptr(labels), float(dloss),
                             _ptr(loss), _ptr(dX), _ptr(dW), _ptr(ws),
                             ws.numel() * ws.element_size(), _stream(stream)), "flce_fused")
@@ -155,6 +272,7 @@ def flce_fused(problem, X, W, labels, dloss, loss, dX, dW, ws, stream=None):
 def flce_count_valid(problem, labels, n_valid, stream=None):
     """n_valid (device int64 [1]) = number of rows whose (shifted) label is
     not the problem's ignore_index."""
+    _check_flce(problem, labels=labels, extra=[("n_valid", n_valid, 1, torch.int64)])
     _check(lib().flce_count_valid(ctypes.byref(problem), _ptr(labels), _ptr(n_valid),
                                   _stream(stream)), "flce_count_valid")
 
@@ -162,6 +280,9 @@ def flce_count_valid(problem, labels, n_valid, stream=None):
 def flce_fused_global(problem, X, W, labels, n_valid_global, dloss, loss, dX, dW, ws,
                       stream=None):
     """flce_fused with the mean's divisor taken from n_valid_global (device int64 [1])."""
+    _check_flce(problem, X=X, W=W, labels=labels, dX=dX, dW=dW,
+                extra=[("loss", loss, 1, torch.float32),
+                       ("n_valid_global", n_valid_global, 1, torch.int64)])
     _check(lib().flce_fused_global(ctypes.byref(problem), _ptr(X), _ptr(W), _ptr(labels),
                                    _ptr(n_valid_global), float(dloss), _ptr(loss), _ptr(dX),
                                    _ptr(dW), _ptr(ws), ws.numel() * ws.element_size(),
@@ -170,9 +291,33 @@ def flce_fused_global(problem, X, W, labels, n_valid_global, dloss, loss, dX, dW
 
 def flce_fused_noalloc(problem, X, W, labels, dloss, loss, dX, dW, stream=None):
     """flce_fused with the library's fixed scratch array instead of a workspace."""
+    _check_flce(problem, X=X, W=W, labels=labels, dX=dX, dW=dW,
+                extra=[("loss", loss, 1, torch.float32)])
     _check(lib().flce_fused_noalloc(ctypes.byref(problem), _ptr(X), _ptr(W), _ptr(labels),
                                     float(dloss), _ptr(loss), _ptr(dX), _ptr(dW),
                                     _stream(stream)), "flce_fused_noalloc")
+
+
+def flce_ce_workspace_size(problem: flce_ce_problem_t, op: int) -> int:
+    return int(lib().flce_ce_workspace_size(ctypes.byref(problem), int(op)))
+
+
+def flce_ce_forward(problem, logits, labels, loss, lse, ws, stream=None):
+    """loss and lse from logits the caller holds (one read of them)."""
+    _check_ce(problem, logits=logits, labels=labels, lse=lse,
+              extra=[("loss", loss, 1, torch.float32)])
+    _check(lib().flce_ce_forward(ctypes.byref(problem), _ptr(logits), _ptr(labels), _ptr(loss),
+                                 _ptr(lse), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "flce_ce_forward")
+
+
+def flce_ce_backward(problem, logits, labels, lse, dloss, dlogits, ws, stream=None):
+    """dlogits from the logits and the forward's lse; dlogits may be logits."""
+    _check_ce(problem, logits=logits, labels=labels, lse=lse, dlogits=dlogits,
+              extra=[("dloss", dloss, 1, torch.float32)])
+    _check(lib().flce_ce_backward(ctypes.byref(problem), _ptr(logits), _ptr(labels), _ptr(lse),
+                                  _ptr(dloss), _ptr(dlogits), _ptr(ws), _nbytes(ws),
+                                  _stream(stream)), "flce_ce_backward")
 
 
 def flce_get_device_status(ws, stream=None):
@@ -189,12 +334,30 @@ def flce_selftest_wait_timeout(ws, limit_ns: int, stream=None) -> None:
            "flce_selftest_wait_timeout")
 
 
+def flce_selftest_approx(x: torch.Tensor) -> torch.Tensor:
+    """[n, 4] fp32: the epilogues' tanh, CUDA's tanhf, the epilogues' exp2,
+    CUDA's exp2f, evaluated on the device at the fp32 CUDA tensor x."""
+    x = x.contiguous()
+    if x.dtype != torch.float32 or not x.is_cuda:
+        raise ValueError("x must be a float32 CUDA tensor")
+    out = torch.empty(x.numel(), 4, dtype=torch.float32, device=x.device)
+    _check(lib().flce_selftest_approx(_ptr(x), x.numel(), _ptr(out), _stream(None)),
+           "flce_selftest_approx")
+    return out
+
+
 def flce_set_schedule(schedule: int) -> int:
     """Set the process-wide flce_fused schedule; returns the previous one."""
     prev = int(lib().flce_set_schedule(int(schedule)))
     if prev < 0:
         raise FlceError(1, "flce_set_schedule")
     return prev
+
+
+def flce_set_workspace_limit(nbytes: int) -> int:
+    """Cap the workspace the automatic flce_fused schedule plans (0 = none);
+    returns the previous cap."""
+    return int(lib().flce_set_workspace_limit(int(nbytes)))
 
 
 def flce_set_wait_limit_ns(ns: int) -> int:
@@ -225,16 +388,34 @@ def flce_kernel_name(kind: int) -> str:
 
 # ----------------------- convenience (allocates outputs) ----------------------
 
-def _problem_of(X, W, ignore_index, softcap, shift_seq_len=0):
+def _problem_of(X, W, ignore_index, softcap, shift_seq_len=0, dX=None, dW=None):
+    """The problem of tensors X [BT, H] and W [V, H], their row strides
+    included (rows must be unit-stride; dX, dW likewise when given)."""
+    if X.dim() != 2 or W.dim() != 2 or X.shape[1] != W.shape[1]:
+        raise ValueError("X must be [BT, H] and W [V, H], got %s and %s"
+                         % (tuple(X.shape), tuple(W.shape)))
+    if X.dtype != W.dtype or X.dtype not in _DTYPES:
+        raise ValueError("X and W must both be bfloat16 or both float32 (got %s, %s)"
+                         % (X.dtype, W.dtype))
     return make_problem(X.shape[0], X.shape[1], W.shape[0], X.dtype, ignore_index, softcap,
-                        shift_seq_len)
+                        shift_seq_len, ldx=_row_stride(X), ldw=_row_stride(W),
+                        lddx=_row_stride(dX) if dX is not None else 0,
+                        lddw=_row_stride(dW) if dW is not None else 0,
+                        dw_fp32=int(dW is not None and dW.dtype == torch.float32))
+
+
+def _ws_for(n, device, where):
+    if n == 0:
+        raise FlceError(1, where)
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def workspace(problem, op, device) -> torch.Tensor:
-    n = flce_workspace_size(problem, op)
-    if n == 0:
-        raise FlceError(1, "flce_workspace_size")
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return _ws_for(flce_workspace_size(problem, op), device, "flce_workspace_size")
+
+
+def ce_workspace(problem, op, device) -> torch.Tensor:
+    return _ws_for(flce_ce_workspace_size(problem, op), device, "flce_ce_workspace_size")
 
 
 def forward(X, W, labels, ignore_index=-100, softcap=0.0, ws=None, stream=None,
@@ -251,25 +432,30 @@ def forward(X, W, labels, ignore_index=-100, softcap=0.0, ws=None, stream=None,
 def backward(X, W, labels, lse, dloss, ignore_index=-100, softcap=0.0, ws=None, stream=None,
              shift_seq_len=0):
     """Return (dX, dW) computed by flce_backward; dloss is a device fp32 tensor."""
-    p = _problem_of(X, W, ignore_index, softcap, shift_seq_len)
+    dX = torch.empty(X.shape, dtype=X.dtype, device=X.device)
+    dW = torch.empty(W.shape, dtype=W.dtype, device=W.device)
+    p = _problem_of(X, W, ignore_index, softcap, shift_seq_len, dX, dW)
     ws = workspace(p, FLCE_OP_BACKWARD, X.device) if ws is None else ws
-    dX = torch.empty_like(X)
-    dW = torch.empty_like(W)
     flce_backward(p, X, W, labels, lse, dloss, dX, dW, ws, stream)
     return dX, dW
 
 
 def fused(X, W, labels, ignore_index=-100, softcap=0.0, dloss=1.0, ws=None, stream=None,
-          n_valid_global=None, shift_seq_len=0):
+          n_valid_global=None, shift_seq_len=0, dX=None, dW=None, dw_fp32=False):
     """Return (loss [1] fp32, dX, dW) computed by flce_fused, or by
     flce_fused_global when n_valid_global (device int64 [1]) is given.
     shift_seq_len = T > 0: labels are token ids of BT/T sequences and the op
-    shifts them itself (position t scored against id t+1)."""
-    p = _problem_of(X, W, ignore_index, softcap, shift_seq_len)
+    shifts them itself (position t scored against id t+1).  X and W may be
+    row-strided views (e.g. a column slice of a wider tensor); dX, dW, when
+    given, receive the gradients (row-strided views allowed), else dense
+    tensors are allocated.  An fp32 dW (given, or dw_fp32=True) is written
+    in fp32 whatever the input type."""
+    dX = torch.empty(X.shape, dtype=X.dtype, device=X.device) if dX is None else dX
+    if dW is None:
+        dW = torch.empty(W.shape, dtype=torch.float32 if dw_fp32 else W.dtype, device=W.device)
+    p = _problem_of(X, W, ignore_index, softcap, shift_seq_len, dX, dW)
     ws = workspace(p, FLCE_OP_FUSED, X.device) if ws is None else ws
     loss = torch.empty(1, dtype=torch.float32, device=X.device)
-    dX = torch.empty_like(X)
-    dW = torch.empty_like(W)
     if n_valid_global is None:
         flce_fused(p, X, W, labels, dloss, loss, dX, dW, ws, stream)
     else:
@@ -284,3 +470,37 @@ def count_valid(X, W, labels, ignore_index=-100, stream=None, shift_seq_len=0) -
     n = torch.empty(1, dtype=torch.int64, device=labels.device)
     flce_count_valid(p, labels, n, stream)
     return n
+
+
+def _ce_problem_of(logits, ignore_index, softcap, shift_seq_len, dlogits=None):
+    if logits.dim() != 2 or logits.dtype not in _DTYPES:
+        raise ValueError("logits must be a 2-D bfloat16 or float32 tensor, got %s %s"
+                         % (logits.dtype, tuple(logits.shape)))
+    return make_ce_problem(logits.shape[0], logits.shape[1], logits.dtype, ignore_index, softcap,
+                           shift_seq_len, ld=_row_stride(logits),
+                           ld_grad=_row_stride(dlogits) if dlogits is not None else 0)
+
+
+def ce_forward(logits, labels, ignore_index=-100, softcap=0.0, ws=None, stream=None,
+               shift_seq_len=0):
+    """Return (loss [1] fp32, lse [BT] fp32) computed by flce_ce_forward from
+    logits [BT, V] (a row-strided view is fine)."""
+    p = _ce_problem_of(logits, ignore_index, softcap, shift_seq_len)
+    ws = ce_workspace(p, FLCE_OP_FORWARD, logits.device) if ws is None else ws
+    loss = torch.empty(1, dtype=torch.float32, device=logits.device)
+    lse = torch.empty(logits.shape[0], dtype=torch.float32, device=logits.device)
+    flce_ce_forward(p, logits, labels, loss, lse, ws, stream)
+    return loss, lse
+
+
+def ce_backward(logits, labels, lse, dloss, ignore_index=-100, softcap=0.0, ws=None,
+                stream=None, shift_seq_len=0, out=None):
+    """Return dlogits computed by flce_ce_backward; dloss is a device fp32
+    [1] tensor.  out: where to write it (pass logits itself to overwrite
+    the logits in place), else a new dense tensor."""
+    out = torch.empty(logits.shape, dtype=logits.dtype, device=logits.device) if out is None \
+        else out
+    p = _ce_problem_of(logits, ignore_index, softcap, shift_seq_len, out)
+    ws = ce_workspace(p, FLCE_OP_BACKWARD, logits.device) if ws is None else ws
+    flce_ce_backward(p, logits, labels, lse, dloss, out, ws, stream)
+    return out

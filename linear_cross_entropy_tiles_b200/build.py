@@ -15,8 +15,9 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT_DIR = os.path.join(HERE, "_build")
 LIB = os.path.join(OUT_DIR, "libflce.so")
-SOURCES = [os.path.join(CSRC, "flce_api.cu"), os.path.join(CSRC, "flce_noalloc.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + [
+SOURCES = [os.path.join(CSRC, "flce_api.cu"), os.path.join(CSRC, "flce_noalloc.cu"),
+           os.path.join(CSRC, "flce_ce.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, "flce.h")]
 
 NVCC_FLAGS = [

@@ -17,17 +17,11 @@
 #include <cstdint>
 
 #include "sm100.cuh"
+#include "ws_header.cuh"
 
 namespace flce {
 
 constexpr int kStatusBadLabel = 5;  // FLCE_ERR_LABEL_OUT_OF_RANGE
-
-// Workspace header, first 256 bytes of every workspace.
-struct WsHeader {
-  int status;
-  int pad;
-  long long n_valid;
-};
 
 __global__ void labels_kernel(const int64_t* __restrict__ labels, int64_t BT, int64_t V,
                               int64_t ignore_index, WsHeader* hdr) {
@@ -263,9 +257,11 @@ __global__ void __launch_bounds__(kLseGradThreads)
 }
 
 // dX rows of a row chunk from its K-split slabs: out = bf16(sum_s slab_s),
-// summed in split order.  n is a multiple of 8.
+// summed in split order.  The slabs are dense rows of H; output rows are
+// ld_out apart.  n (rows * H) and H are multiples of 8, as is ld_out.
 __global__ void slab_reduce_kernel(const float* __restrict__ slabs, int n_slabs,
-                                   int64_t slab_stride, int64_t n, __nv_bfloat16* __restrict__ out,
+                                   int64_t slab_stride, int64_t n, int64_t H,
+                                   __nv_bfloat16* __restrict__ out, int64_t ld_out,
                                    const WsHeader* hdr) {
   if (hdr->status != 0) return;
   for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < n;
@@ -281,7 +277,7 @@ __global__ void slab_reduce_kernel(const float* __restrict__ slabs, int n_slabs,
     }
     __nv_bfloat162 h[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
                            __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
-    *reinterpret_cast<uint4*>(out + i) = *reinterpret_cast<uint4*>(h);
+    *reinterpret_cast<uint4*>(out + (i / H) * ld_out + i % H) = *reinterpret_cast<uint4*>(h);
   }
 }
 
@@ -323,6 +319,7 @@ struct SimtEpi {
   const int64_t* labels;
   int64_t ignore_index;
   int64_t BT, H, V;
+  int64_t ldx, ldw, lddx, lddw;  // row strides of X, W, dX, dW (elements)
   float softcap;
   // logits modes
   float2* partial;         // [ceil(V/32)][BT]
@@ -358,8 +355,8 @@ __global__ void simt_logits_kernel(const T* __restrict__ X, const T* __restrict_
     for (int i = 0; i < 4; ++i) {
       const int rr = ty + 8 * i;
       const int64_t xr = m0 + rr, wr = ep.v0 + n0 + rr, kk = k0 + tx;
-      xs[rr][tx] = (xr < ep.BT && kk < ep.H) ? ld_f(X + xr * ep.H + kk) : 0.f;
-      ws[rr][tx] = (wr < ep.V && kk < ep.H) ? ld_f(W + wr * ep.H + kk) : 0.f;
+      xs[rr][tx] = (xr < ep.BT && kk < ep.H) ? ld_f(X + xr * ep.ldx + kk) : 0.f;
+      ws[rr][tx] = (wr < ep.V && kk < ep.H) ? ld_f(W + wr * ep.ldw + kk) : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -427,12 +424,12 @@ __global__ void simt_gemm_kernel(const T* __restrict__ Bsrc, SimtEpi ep) {
         as[rr][tx] = (gr < ep.BT && gc < ep.chunk) ? ep.G[gr * ep.ldg + gc] : 0.f;
         const int64_t wr = k0 + rr, wc = n0 + tx;  // W[v0 + wr][wc]
         bs[rr][tx] = (wr < ep.chunk && ep.v0 + wr < ep.V && wc < ep.H)
-                         ? ld_f(Bsrc + (ep.v0 + wr) * ep.H + wc) : 0.f;
+                         ? ld_f(Bsrc + (ep.v0 + wr) * ep.ldw + wc) : 0.f;
       } else {
         const int64_t gk = k0 + rr, gm = m0 + tx;  // G[gk][gm] is A[gm][gk]
         as[tx][rr] = (gk < ep.BT && gm < ep.chunk) ? ep.G[gk * ep.ldg + gm] : 0.f;
         const int64_t xr = k0 + rr, xc = n0 + tx;
-        bs[rr][tx] = (xr < ep.BT && xc < ep.H) ? ld_f(Bsrc + xr * ep.H + xc) : 0.f;
+        bs[rr][tx] = (xr < ep.BT && xc < ep.H) ? ld_f(Bsrc + xr * ep.ldx + xc) : 0.f;
       }
     }
     __syncthreads();
@@ -457,10 +454,10 @@ __global__ void simt_gemm_kernel(const T* __restrict__ Bsrc, SimtEpi ep) {
       if (!ep.dx_last)
         *p = a;
       else
-        static_cast<T*>(ep.dx)[row * ep.H + col] = from_f<T>(a);
+        static_cast<T*>(ep.dx)[row * ep.lddx + col] = from_f<T>(a);
     } else {
       const int64_t v = ep.v0 + row;
-      if (v < ep.V) static_cast<T*>(ep.dw)[v * ep.H + col] = from_f<T>(acc[i]);
+      if (v < ep.V) static_cast<T*>(ep.dw)[v * ep.lddw + col] = from_f<T>(acc[i]);
     }
   }
 }

@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 
 #include "flce.h"
+#include "internal.h"
 #include "aux_kernels.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
@@ -41,15 +42,24 @@ thread_local int32_t t_launches = 0;
 enum Kind : int32_t {
   K_LABELS = 0, K_LSE_GEMM, K_COMBINE, K_FINALIZE, K_GRAD_GEMM, K_DX_GEMM, K_DW_GEMM,
   K_SIMT_LOGITS, K_SIMT_GRAD, K_SIMT_DX, K_SIMT_DW, K_MEMSET, K_LSEP_GEMM, K_LSE_GRAD,
-  K_DWACC_GEMM, K_DX_REDUCE, K_COUNT_VALID, K_SET_NVALID, K_SHIFT_LABELS, K_NUM_KINDS
+  K_DWACC_GEMM, K_DX_REDUCE, K_COUNT_VALID, K_SET_NVALID, K_SHIFT_LABELS,
+  // launched from flce_ce.cu (kinds fixed in internal.h)
+  K_CE_FORWARD, K_CE_BACKWARD, K_CE_FUSED, K_NUM_KINDS
 };
+static_assert(int32_t(K_CE_FORWARD) == int32_t(flce_internal::kKindCeForward) &&
+                  int32_t(K_CE_BACKWARD) == int32_t(flce_internal::kKindCeBackward) &&
+                  int32_t(K_CE_FUSED) == int32_t(flce_internal::kKindCeFused),
+              "kernel kinds shared with flce_ce.cu");
 const char* const kKindNames[K_NUM_KINDS] = {
     "labels", "lse_gemm", "lse_combine", "loss_finalize", "grad_gemm", "dx_gemm", "dw_gemm",
     "simt_lse", "simt_grad", "simt_dx", "simt_dw", "memset", "lse_p_gemm", "lse_grad",
-    "dw_acc_gemm", "dx_reduce", "count_valid", "set_n_valid", "shift_labels"};
+    "dw_acc_gemm", "dx_reduce", "count_valid", "set_n_valid", "shift_labels", "ce_forward",
+    "ce_backward", "ce_fused"};
 
 // flce_fused schedule: 0 = choose, 1 = two-pass recompute, 2 = fused-in-forward.
 std::atomic<int32_t> g_schedule{0};
+// Cap on the workspace the automatic schedule may plan (0 = none).
+std::atomic<unsigned long long> g_ws_limit{0};
 
 // Optional per-launch CUDA-event timing (flce_profile_start / _stop).
 struct Profiler {
@@ -82,6 +92,8 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 struct Plan {
   int64_t BT = 0, H = 0, V = 0;
+  int64_t ldx = 0, ldw = 0, lddx = 0, lddw = 0;  // row strides (elements) of X, W, dX, dW
+  bool dw_f32 = false;    // bf16 inputs with an fp32 dW (the fused schedule sums into dW)
   size_t off_shift = 0;   // shifted labels [BT] int64 when the op shifts token ids
   bool tc = false;        // bf16 tensor-core path (else fp32 SIMT)
   int bn = 256;           // N tile of the logit GEMMs and of dX / dW
@@ -105,13 +117,23 @@ bool softcap_on(float c) { return c > 0.f && std::isfinite(c); }
 
 flce_status_t check_problem(const flce_problem_t* p) {
   if (!p) return FLCE_ERR_INVALID_ARG;
-  if (p->reserved1 != 0 || p->shift_seq_len < 0) return FLCE_ERR_INVALID_ARG;
+  if ((p->dw_fp32 != 0 && p->dw_fp32 != 1) || p->shift_seq_len < 0) return FLCE_ERR_INVALID_ARG;
   if (p->shift_seq_len > 0 && p->BT % p->shift_seq_len != 0) return FLCE_ERR_INVALID_ARG;
   if (p->BT < 0 || p->H <= 0 || p->V <= 0) return FLCE_ERR_INVALID_ARG;
   if (p->dtype != FLCE_BF16 && p->dtype != FLCE_FP32) return FLCE_ERR_UNSUPPORTED;
   if (p->H % 8 != 0) return FLCE_ERR_MISALIGNED;
   if (p->BT >= (int64_t(1) << 31) || p->V >= (int64_t(1) << 31) || p->H >= (int64_t(1) << 31))
     return FLCE_ERR_UNSUPPORTED;
+  // Row strides: 0 = H; at least H; rows on 16-byte boundaries.
+  const int64_t esz = p->dtype == FLCE_BF16 ? 2 : 4;
+  const int64_t dw_esz = p->dw_fp32 ? 4 : esz;
+  const int64_t lds[4] = {p->ldx, p->ldw, p->lddx, p->lddw};
+  for (int i = 0; i < 4; ++i) {
+    const int64_t ld = lds[i];
+    if (ld < 0 || (ld != 0 && ld < p->H)) return FLCE_ERR_INVALID_ARG;
+    if (ld >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+    if ((ld * (i == 3 ? dw_esz : esz)) % 16 != 0) return FLCE_ERR_MISALIGNED;
+  }
   // Tile ids are 32-bit: the largest grid (BT x V logits in 128 x 256 tiles,
   // up to 8 K splits) must stay below 2^31 work units.
   const int64_t bt_tiles = (p->BT + 127) / 128, v_tiles = (p->V + 255) / 256;
@@ -207,7 +229,8 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl) {
   off = align256(off + size_t(pl->part_tiles) * rows * 8);
   pl->off_p = off;
   off = align256(off + size_t(pl->Cb) * size_t(pl->ldp) * 2);
-  if (pl->n_row_chunks > 1) {
+  // The fp32 running sum of dW over row chunks, unless dW itself is fp32.
+  if (pl->n_row_chunks > 1 && !p->dw_fp32) {
     pl->off_dwacc = off;
     off = align256(off + size_t(V) * size_t(H) * 4);
   }
@@ -221,23 +244,43 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl) {
   pl->total = off;
 }
 
-void make_plan_base(const flce_problem_t* p, int op, Plan* pl);
+void make_plan_base(const flce_problem_t* p, int op, Plan* pl, int64_t vc_max);
+
+int64_t eff_ld(int64_t ld, int64_t H) { return ld == 0 ? H : ld; }
 
 // Every schedule's plan, plus room for the shifted labels when the op
-// shifts token ids itself.
+// shifts token ids itself.  Under the automatic schedule with a workspace
+// cap, flce_fused takes the fused-in-forward plan only if it fits, else the
+// recompute plan with the widest vocabulary chunk that fits.
 void make_plan(const flce_problem_t* p, int op, Plan* pl) {
-  make_plan_base(p, op, pl);
+  const size_t extra = p->shift_seq_len > 0 ? align256(size_t(p->BT) * 8) : 0;
+  const unsigned long long limit = g_schedule.load() == 0 ? g_ws_limit.load() : 0ull;
+  make_plan_base(p, op, pl, 32768);
+  if (limit && op == FLCE_OP_FUSED && p->dtype == FLCE_BF16 && pl->total + extra > limit) {
+    for (int64_t vc = 32768; vc >= 256; vc /= 2) {
+      *pl = Plan{};
+      make_plan_base(p, FLCE_OP_FUSED + 16, pl, vc);  // the fused op, recompute schedule
+      if (pl->total + extra <= limit) break;
+    }
+  }
+  pl->dw_f32 = p->dw_fp32 && p->dtype == FLCE_BF16;
+  pl->ldx = eff_ld(p->ldx, p->H);
+  pl->ldw = eff_ld(p->ldw, p->H);
+  pl->lddx = eff_ld(p->lddx, p->H);
+  pl->lddw = eff_ld(p->lddw, p->H);
   if (p->shift_seq_len > 0) {
     pl->off_shift = pl->total;
     pl->total = align256(pl->total + size_t(p->BT) * 8);
   }
 }
 
-void make_plan_base(const flce_problem_t* p, int op, Plan* pl) {
+// op FLCE_OP_FUSED + 16 (internal): the fused op on the recompute schedule.
+void make_plan_base(const flce_problem_t* p, int op, Plan* pl, int64_t vc_max) {
   if (op == FLCE_OP_FUSED && use_fused_forward(p)) {
     make_plan_fused_forward(p, pl);
     return;
   }
+  if (op == FLCE_OP_FUSED + 16) op = FLCE_OP_FUSED;
   pl->BT = p->BT;
   pl->H = p->H;
   pl->V = p->V;
@@ -249,11 +292,13 @@ void make_plan_base(const flce_problem_t* p, int op, Plan* pl) {
     pl->bn = 256;
     pl->part_shift = partial_shift(H);
     pl->part_tiles = cdiv(V, int64_t(1) << pl->part_shift);
-    // Chunk width: G_c (BT x Vc bf16) kept at <= 512 MiB, Vc in [1024, 32768].
+    // Chunk width: G_c (BT x Vc bf16) kept at <= 512 MiB, Vc in [1024, 32768]
+    // (narrower only under a workspace cap).
     int64_t vc = (int64_t(1) << 29) / (2 * (BT > 0 ? BT : 1));
     vc = vc / 256 * 256;
     if (vc < 1024) vc = 1024;
     if (vc > 32768) vc = 32768;
+    if (vc > vc_max) vc = vc_max;
     pl->Vc = vc < round_up(V, 256) ? vc : round_up(V, 256);
     pl->g_elem = 2;
   } else {
@@ -482,6 +527,9 @@ TcEpi base_epi(const flce_problem_t* p, const Plan& pl, const Ptrs& q) {
   e.V = pl.V;
   e.H = pl.H;
   e.softcap = softcap_on(p->softcap) ? p->softcap : 0.f;
+  e.ld_dx = pl.lddx;
+  e.ld_dw = pl.lddw;
+  e.ld_acc = pl.H;
   return e;
 }
 
@@ -494,6 +542,10 @@ SimtEpi base_simt(const flce_problem_t* p, const Plan& pl, const Ptrs& q) {
   e.H = pl.H;
   e.V = pl.V;
   e.softcap = softcap_on(p->softcap) ? p->softcap : 0.f;
+  e.ldx = pl.ldx;
+  e.ldw = pl.ldw;
+  e.lddx = pl.lddx;
+  e.lddw = pl.lddw;
   return e;
 }
 
@@ -555,8 +607,8 @@ flce_status_t enqueue_forward(const flce_problem_t* p, const Plan& pl, const Ptr
   if (BT > 0) {
     if (pl.tc) {
       CUtensorMap ma, mb;
-      if (!make_map(&ma, q.X, H, BT, H * 2, 64, kBM)) return FLCE_ERR_CUDA;
-      if (!make_map(&mb, q.W, H, V, H * 2, 64, b_box_rows())) return FLCE_ERR_CUDA;
+      if (!make_map(&ma, q.X, H, BT, pl.ldx * 2, 64, kBM)) return FLCE_ERR_CUDA;
+      if (!make_map(&mb, q.W, H, V, pl.ldw * 2, 64, b_box_rows())) return FLCE_ERR_CUDA;
       TcEpi ep = base_epi(p, pl, q);
       ep.partial = partial;
       ep.target = target;
@@ -592,10 +644,10 @@ flce_status_t enqueue_forward(const flce_problem_t* p, const Plan& pl, const Ptr
 flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Ptrs& q,
                                cudaStream_t st) {
   const int64_t BT = pl.BT, V = pl.V, H = pl.H;
-  const size_t esz = pl.tc ? 2 : 4;
+  const size_t esz = (pl.tc && !pl.dw_f32) ? 2 : 4;  // dW's element size
   if (BT == 0) {
     prof_before(st);
-    FLCE_TRY(cudaMemsetAsync(q.dW, 0, size_t(V) * size_t(H) * esz, st));
+    FLCE_TRY(cudaMemset2DAsync(q.dW, size_t(pl.lddw) * esz, 0, size_t(H) * esz, size_t(V), st));
     prof_after(st, K_MEMSET);
     return FLCE_OK;
   }
@@ -605,13 +657,13 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
     __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(q.ws + pl.off_g);
     CUtensorMap mx_k, mw_k, mg_k, mw_mn, mg_mn, mx_mn, mg_out, mdx_out;
     bool ok = make_map(&mg_out, G, pl.ldg, BT, pl.ldg * 2, 64, 32) &&
-              make_map(&mdx_out, q.dX, H, BT, H * 2, 64, 32) &&
-              make_map(&mx_k, q.X, H, BT, H * 2, 64, kBM) &&
-              make_map(&mw_k, q.W, H, V, H * 2, 64, b_box_rows()) &&
+              make_map(&mdx_out, q.dX, H, BT, pl.lddx * 2, 64, 32) &&
+              make_map(&mx_k, q.X, H, BT, pl.ldx * 2, 64, kBM) &&
+              make_map(&mw_k, q.W, H, V, pl.ldw * 2, 64, b_box_rows()) &&
               make_map(&mg_k, G, pl.ldg, BT, pl.ldg * 2, 64, kBM) &&
-              make_map(&mw_mn, q.W, H, V, H * 2, 64, 64) &&
+              make_map(&mw_mn, q.W, H, V, pl.ldw * 2, 64, 64) &&
               make_map(&mg_mn, G, pl.ldg, BT, pl.ldg * 2, 64, 64) &&
-              make_map(&mx_mn, q.X, H, BT, H * 2, 64, 64);
+              make_map(&mx_mn, q.X, H, BT, pl.ldx * 2, 64, 64);
     if (!ok) return FLCE_ERR_CUDA;
     const int sms = device_sms();
     for (int64_t c = 0; c < pl.n_chunks; ++c) {
@@ -648,10 +700,16 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
       FLCE_TRY((launch_gemm<false, true, EPI_DX>(mg_k, mw_mn, mdx_out, gx, ex, sms, st)));
       // dW_c = G_c^T X     (K = BT); the output map ends at the chunk's last row
       CUtensorMap mdw_out;
-      if (!make_map(&mdw_out, q.dW, H, v0 + width, H * 2, 64, 32)) return FLCE_ERR_CUDA;
+      const bool ok_dw =
+          pl.dw_f32 ? make_map(&mdw_out, q.dW, H, v0 + width, pl.lddw * 4, 32, 32,
+                               CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+                    : make_map(&mdw_out, q.dW, H, v0 + width, pl.lddw * 2, 64, 32);
+      if (!ok_dw) return FLCE_ERR_CUDA;
       TcEpi ewo = ep;
       ewo.out_row_off = int(v0);
       ewo.out_cols = int(H);
+      ewo.out_f32 = pl.dw_f32 ? 1 : 0;
+      ewo.dw32 = static_cast<float*>(q.dW);
       GemmArgs gw{width, H, BT, false};
       FLCE_TRY((launch_gemm<true, true, EPI_DW>(mg_mn, mx_mn, mdw_out, gw, ewo, sms, st)));
     }
@@ -713,11 +771,15 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
   float* lse = reinterpret_cast<float*>(q.ws + pl.off_lse);
   __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(q.ws + pl.off_p);
   CUtensorMap mx_k, mw_k, mw_mn, mx_mn, mdw_out;
-  if (!(make_map(&mdw_out, q.dW, H, V, H * 2, 64, 32) &&
-        make_map(&mx_k, q.X, H, BT, H * 2, 64, kBM) &&
-        make_map(&mw_k, q.W, H, V, H * 2, 64, b_box_rows()) &&
-        make_map(&mw_mn, q.W, H, V, H * 2, 64, 64) &&
-        make_map(&mx_mn, q.X, H, BT, H * 2, 64, 64)))
+  // dW's map: bf16 pieces of 64 columns, or fp32 pieces of 32 when dW is fp32
+  const bool ok_dw = pl.dw_f32 ? make_map(&mdw_out, q.dW, H, V, pl.lddw * 4, 32, 32,
+                                          CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+                               : make_map(&mdw_out, q.dW, H, V, pl.lddw * 2, 64, 32);
+  if (!(ok_dw &&
+        make_map(&mx_k, q.X, H, BT, pl.ldx * 2, 64, kBM) &&
+        make_map(&mw_k, q.W, H, V, pl.ldw * 2, 64, b_box_rows()) &&
+        make_map(&mw_mn, q.W, H, V, pl.ldw * 2, 64, 64) &&
+        make_map(&mx_mn, q.X, H, BT, pl.ldx * 2, 64, 64)))
     return FLCE_ERR_CUDA;
   const int sms = device_sms();
   const float cap = softcap_on(p->softcap) ? p->softcap : 0.f;
@@ -728,8 +790,8 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     if (!(make_map(&mp_k, P, pl.ldp, rows, pl.ldp * 2, 64, kBM) &&
           make_map(&mp_mn, P, pl.ldp, rows, pl.ldp * 2, 64, 64) &&
           make_map(&mp_out, P, pl.ldp, rows, pl.ldp * 2, 64, 32) &&
-          make_map(&mdx_out, static_cast<__nv_bfloat16*>(q.dX) + row0 * H, H, rows, H * 2, 64,
-                   32)))
+          make_map(&mdx_out, static_cast<__nv_bfloat16*>(q.dX) + row0 * pl.lddx, H, rows,
+                   pl.lddx * 2, 64, 32)))
       return FLCE_ERR_CUDA;
     TcEpi ep = base_epi(p, pl, q);
     ep.partial = partial;
@@ -753,7 +815,7 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     FLCE_TRY(cudaGetLastError());
     // dX rows of this chunk: K runs over the whole vocabulary
     TcEpi ex = ep;
-    ex.dx = static_cast<__nv_bfloat16*>(q.dX) + row0 * H;
+    ex.dx = static_cast<__nv_bfloat16*>(q.dX) + row0 * pl.lddx;
     ex.dx_first = 1;
     ex.dx_last = 1;
     ex.dx_acc = reinterpret_cast<float*>(q.ws + pl.off_dxslab);
@@ -767,23 +829,28 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
       int blocks = int(cdiv(n, 8 * 256));
       if (blocks > 8 * sms) blocks = 8 * sms;
       prof_before(st);
-      slab_reduce_kernel<<<blocks, 256, 0, st>>>(ex.dx_acc, pl.dx_splits, ex.slab_stride, n,
-                                                 ex.dx, hdr);
+      slab_reduce_kernel<<<blocks, 256, 0, st>>>(ex.dx_acc, pl.dx_splits, ex.slab_stride, n, H,
+                                                 ex.dx, pl.lddx, hdr);
       prof_after(st, K_DX_REDUCE);
       FLCE_TRY(cudaGetLastError());
     }
-    // dW += G_b^T X_b
+    // dW += G_b^T X_b: an fp32 running sum over the row chunks, in the
+    // workspace, or in dW itself when dW is fp32
     TcEpi ew = ep;
-    ew.dx_acc = reinterpret_cast<float*>(q.ws + pl.off_dwacc);
+    ew.dx_acc = pl.dw_f32 ? static_cast<float*>(q.dW)
+                          : reinterpret_cast<float*>(q.ws + pl.off_dwacc);
+    ew.ld_acc = pl.dw_f32 ? pl.lddw : H;
+    ew.out_f32 = pl.dw_f32 ? 1 : 0;
     ew.dx = static_cast<__nv_bfloat16*>(q.dW);
+    ew.ld_dx = pl.lddw;
     ew.dx_first = b == 0;
     ew.dx_last = b == pl.n_row_chunks - 1;
     ew.out_cols = int(H);
-    // The sum goes out by TMA stores: fp32 rows of the running sum, or the
-    // bf16 dW on the last chunk.
+    // The sum goes out by TMA stores: fp32 rows of the running sum, then dW
+    // on the last chunk (bf16, or the fp32 sum itself).
     ew.tma_rmw = 1;
     CUtensorMap macc;
-    if (!ew.dx_last && !make_map(&macc, ew.dx_acc, H, V, H * 4, 32, 32,
+    if (!ew.dx_last && !make_map(&macc, ew.dx_acc, H, V, size_t(ew.ld_acc) * 4, 32, 32,
                                  CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
       return FLCE_ERR_CUDA;
     GemmArgs gw{V, H, rows, false};
@@ -799,6 +866,20 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
 
 bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
 
+// The epilogues' own approximations beside CUDA's functions, for a bound
+// test: out[4i..4i+3] = tanh_fast(x), tanhf(x), ex2a(x), exp2f(x).
+__global__ void approx_selftest_kernel(const float* __restrict__ x, int64_t n,
+                                       float* __restrict__ out) {
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const float v = x[i];
+    out[4 * i] = tanh_fast(v);
+    out[4 * i + 1] = tanhf(v);
+    out[4 * i + 2] = ex2a(v);
+    out[4 * i + 3] = exp2f(v);
+  }
+}
+
 flce_status_t check_common(const flce_problem_t* p, const void* X, const void* W,
                            const int64_t* labels, void* ws) {
   if (p->BT > 0 && (!X || !labels)) return FLCE_ERR_INVALID_ARG;
@@ -809,6 +890,43 @@ flce_status_t check_common(const flce_problem_t* p, const void* X, const void* W
 }
 
 }  // namespace
+
+// ------------------------- shared with flce_ce.cu ---------------------------
+
+namespace flce_internal {
+
+void prof_before(cudaStream_t st) { ::prof_before(st); }
+void prof_after(cudaStream_t st, int32_t kind) { ::prof_after(st, kind); }
+void reset_launch_count() { t_launches = 0; }
+
+cudaError_t launch_labels(const int64_t* labels, int64_t BT, int64_t V, int64_t ignore_index,
+                          void* ws, cudaStream_t st) {
+  ::prof_before(st);
+  labels_kernel<<<1, 1024, 0, st>>>(labels, BT, V, ignore_index, static_cast<WsHeader*>(ws));
+  ::prof_after(st, K_LABELS);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_shift(const int64_t* ids, int64_t BT, int64_t T, int64_t ignore_index,
+                         int64_t* out, cudaStream_t st) {
+  if (BT <= 0) return cudaSuccess;
+  int blocks = int(cdiv(BT, 256));
+  if (blocks > 1024) blocks = 1024;
+  ::prof_before(st);
+  shift_labels_kernel<<<blocks, 256, 0, st>>>(ids, BT, T, ignore_index, out);
+  ::prof_after(st, K_SHIFT_LABELS);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const float* row_loss, int64_t BT, const void* ws, float* loss,
+                            cudaStream_t st) {
+  ::prof_before(st);
+  finalize_kernel<<<1, 1024, 0, st>>>(row_loss, BT, static_cast<const WsHeader*>(ws), loss);
+  ::prof_after(st, K_FINALIZE);
+  return cudaGetLastError();
+}
+
+}  // namespace flce_internal
 
 // ------------------------------- C ABI -------------------------------------
 
@@ -957,6 +1075,19 @@ flce_status_t flce_selftest_wait_timeout(void* ws, uint64_t limit_ns, struct CUs
   selftest_wait_kernel<<<1, 32, 0, st>>>(hdr, limit_ns);
   return cuda_status(cudaGetLastError());
 }
+
+flce_status_t flce_selftest_approx(const float* x, int64_t n, float* out, struct CUstream_st* stream) {
+  if (n < 0 || (n > 0 && (!x || !out))) return FLCE_ERR_INVALID_ARG;
+  if (!aligned(x, 4) || !aligned(out, 4)) return FLCE_ERR_MISALIGNED;
+  if (n == 0) return FLCE_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int blocks = int(cdiv(n, 256));
+  if (blocks > 4096) blocks = 4096;
+  approx_selftest_kernel<<<blocks, 256, 0, st>>>(x, n, out);
+  return cuda_status(cudaGetLastError());
+}
+
+uint64_t flce_set_workspace_limit(uint64_t bytes) { return g_ws_limit.exchange(bytes); }
 
 int32_t flce_set_schedule(int32_t schedule) {
   if (schedule < FLCE_SCHEDULE_AUTO || schedule > FLCE_SCHEDULE_FUSED_FORWARD) return -1;

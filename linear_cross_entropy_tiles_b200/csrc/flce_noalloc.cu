@@ -11,9 +11,10 @@
 //
 // The array is shared by every call on a device and keeps whatever the last
 // call left in it.  The fused computation writes every scratch byte it later
-// reads within the same call (the status word, N_valid, the LSE partials, the
-// G chunk and the dX accumulator), so nothing has to be cleared between
-// calls.  Two calls whose GPU work overlaps in time (different streams, or
+// reads within the same call (the status word, N_valid, the shifted labels,
+// the LSE partials, the q / G chunk, the dX accumulator or split slabs, and
+// the dW running sum, whose first row chunk stores without reading), so
+// nothing has to be cleared between calls.  Two calls whose GPU work overlaps in time (different streams, or
 // different host threads on the same device) race on the array and give
 // wrong results; serialise them.
 #include <mutex>
@@ -30,20 +31,26 @@ static __device__ __align__(256) unsigned char g_scratch[FLCE_NOALLOC_SCRATCH_BY
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
+bool g_looked_up[kMaxDevices] = {};
 
-// Device address of g_scratch on the current device, looked up once per
-// device (the first call on each device does it).
-flce_status_t scratch_address(void** out) {
+// Device address of g_scratch in the current device's context.  It is looked
+// up on every call (cheap once the module is loaded), so a context that was
+// torn down and made again, e.g. by cudaDeviceReset, never sees a stale
+// address.  The first look-up on a device may load the module; it is refused
+// while `st` is being captured into a graph, where loading is not allowed.
+flce_status_t scratch_address(cudaStream_t st, void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FLCE_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return FLCE_ERR_CUDA;
-    g_addr[dev] = p;
+  if (!g_looked_up[dev]) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return FLCE_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return FLCE_ERR_INVALID_ARG;
   }
-  *out = g_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return FLCE_ERR_CUDA;
+  g_looked_up[dev] = true;
+  *out = p;
   return FLCE_OK;
 }
 
@@ -57,7 +64,7 @@ extern "C" FLCE_API flce_status_t flce_fused_noalloc(const flce_problem_t* p, co
   if (need == 0) return FLCE_ERR_INVALID_ARG;
   if (need > size_t(FLCE_NOALLOC_SCRATCH_BYTES)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
   void* ws = nullptr;
-  flce_status_t s = scratch_address(&ws);
+  flce_status_t s = scratch_address(reinterpret_cast<cudaStream_t>(stream), &ws);
   if (s != FLCE_OK) return s;
   return flce_fused(p, X, W, labels, dloss, loss, dX, dW, ws, size_t(FLCE_NOALLOC_SCRATCH_BYTES),
                     stream);

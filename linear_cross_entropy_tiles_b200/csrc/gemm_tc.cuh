@@ -94,6 +94,14 @@ struct TcEpi {
   int dx_first, dx_last;
   // EPI_DW
   __nv_bfloat16* dw;        // [V][H]
+  // Row strides (elements) of dx and dw where the epilogue stores them
+  // itself rather than through a TMA map, and of the fp32 running sum dx_acc.
+  int64_t ld_dx, ld_dw, ld_acc;
+  // 1: the result is fp32 -- EPI_DW stores fp32 pieces (through an fp32 map,
+  // or to dw32 without one); a running sum's last pass stores the fp32 sum
+  // (to dx_acc, which then is the output) instead of converting it.
+  int out_f32;
+  float* dw32;
   // EPI_LSE_P (fused-in-forward schedule): rows of this launch start at row0;
   // P is the chunk buffer [rows][ldp] of exp(y - reference), bf16
   int64_t row0;
@@ -415,7 +423,7 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
   // K-split partial: fp32 into this split's slab; a reduction kernel sums them.
   float* slab = ep.dx_acc + int64_t(split) * ep.slab_stride + row * ep.H;
   // Otherwise a running sum in fp32 (streamed: read and written once per launch).
-  float* accrow = ep.dx_acc + row * ep.H;
+  float* accrow = ep.dx_acc + row * ep.ld_acc;
 #pragma unroll 1
   for (int gq = c_lo * 32 / kLoadCols; gq < c_hi * 32 / kLoadCols; ++gq) {
     uint32_t vg[kLoadCols];
@@ -426,6 +434,13 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
       const int c = gq * (kLoadCols / 32) + cc;
       const uint32_t* v = vg + cc * 32;
       if (direct) {
+        if (ep.out_f32) {
+          float a[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(v[k]);
+          put_f32(tma, c, a);
+          continue;
+        }
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -449,7 +464,7 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
           a[4 * g + 2] = __uint_as_float(v[4 * g + 2]) + pv.z;
           a[4 * g + 3] = __uint_as_float(v[4 * g + 3]) + pv.w;
         }
-        if (!ep.dx_last) {
+        if (!ep.dx_last || ep.out_f32) {
           put_f32(tma, c, a);
         } else {
           uint32_t packed[16];
@@ -487,10 +502,10 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
                                      __uint_as_float(v[4 * g + 1]) + prev[g].y,
                                      __uint_as_float(v[4 * g + 2]) + prev[g].z,
                                      __uint_as_float(v[4 * g + 3]) + prev[g].w);
-        if (!ep.dx_last) {
+        if (!ep.dx_last || ep.out_f32) {
           __stcs(reinterpret_cast<float4*>(accrow + col), a);
         } else {
-          *reinterpret_cast<uint2*>(ep.dx + row * ep.H + col) =
+          *reinterpret_cast<uint2*>(ep.dx + row * ep.ld_dx + col) =
               make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
         }
       }
@@ -516,6 +531,13 @@ __device__ __forceinline__ void epi_dw(const TcEpi& ep, const TcShape& sh, int m
       const int c = gq * (kLoadCols / 32) + cc;
       const uint32_t* v = vg + cc * 32;
       if (tma) {
+        if (ep.out_f32) {
+          float a[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(v[k]);
+          put_f32(tma, c, a);
+          continue;
+        }
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -529,7 +551,13 @@ __device__ __forceinline__ void epi_dw(const TcEpi& ep, const TcShape& sh, int m
         const int64_t col = int64_t(n0) + c * 32 + g8 * 8;
         if (col >= ep.H) break;
         const uint32_t* u = v + g8 * 8;
-        *reinterpret_cast<uint4*>(ep.dw + vrow * ep.H + col) = make_uint4(
+        if (ep.out_f32) {
+          float* d = ep.dw32 + vrow * ep.ld_dw + col;
+          *reinterpret_cast<uint4*>(d) = make_uint4(u[0], u[1], u[2], u[3]);
+          *reinterpret_cast<uint4*>(d + 4) = make_uint4(u[4], u[5], u[6], u[7]);
+          continue;
+        }
+        *reinterpret_cast<uint4*>(ep.dw + vrow * ep.ld_dw + col) = make_uint4(
             pack_bf16x2(__uint_as_float(u[0]), __uint_as_float(u[1])),
             pack_bf16x2(__uint_as_float(u[2]), __uint_as_float(u[3])),
             pack_bf16x2(__uint_as_float(u[4]), __uint_as_float(u[5])),

@@ -53,6 +53,49 @@ WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class CEWorkload:
+    """Logits a caller already holds, for the cross-entropy-only path."""
+    name: str
+    BT: int
+    V: int
+    dtype: str
+    std: float          # logits ~ N(0, std^2), rounded to dtype
+    ignore_frac: float
+    softcap: float
+    seed: int
+
+    @property
+    def bytes_per_step(self) -> float:
+        """Algorithmic HBM bytes of forward + backward: the logits read twice
+        and the gradient written once (labels and lse are negligible)."""
+        return 3.0 * self.BT * self.V * (2 if self.dtype == "bf16" else 4)
+
+
+# PyTorch PR #126348's llm.c tensor: batch 32, sequence 1024, vocabulary
+# 50257, bf16.  The logits' scale is that of the GPT-2 LM head above: with
+# X ~ N(0, 1) and W ~ N(0, 0.02^2) over H = 768, X W^T has standard deviation
+# 0.02 * sqrt(768).
+CE_WORKLOADS = {
+    "ce_llmc": CEWorkload("ce_llmc", 32 * 1024, 50257, "bf16", 0.02 * 768 ** 0.5, 0.0, 0.0, 21),
+}
+
+
+def make_ce_workload(w: CEWorkload, device="cpu"):
+    """Return (logits [BT, V], labels int64 [BT]) of a CE workload: normal
+    draws times std rounded (RNE) to dtype, labels uniform in [0, V), an
+    exact fraction of rows ignored (seeded permutation)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(w.seed))
+    Z = (torch.randn(w.BT, w.V, generator=g, device=device, dtype=torch.float32)
+         * w.std).to(torch_dtype(w.dtype))
+    labels = torch.randint(0, w.V, (w.BT,), generator=g, device=device, dtype=torch.int64)
+    n_ignore = int(round(w.ignore_frac * w.BT))
+    if n_ignore:
+        labels[torch.randperm(w.BT, generator=g, device=device)[:n_ignore]] = IGNORE_INDEX
+    return Z, labels
+
+
 def ragged_bt_list() -> list[int]:
     """The 82 BT values of the ragged sweep, drawn with numpy's legacy seed 0
     (the issue gives the formula but no seed)."""

@@ -22,7 +22,7 @@ def built():
 def test_exports_every_declared_symbol():
     header = open(os.path.join(ROOT, "include", "flce.h")).read()
     declared = re.findall(r"FLCE_API\s+[\w\s\*]+?\b(flce_\w+)\s*\(", header)
-    assert len(declared) == 16
+    assert len(declared) == 21
     assert set(declared) == set(binding.EXPORTS)
     lib = binding.lib()
     for name in declared:
@@ -128,7 +128,7 @@ def test_problem_checks_before_any_launch():
         assert L.flce_fused(ctypes.byref(p), A, A, A, 1.0, A, A, A, A, 1 << 40, None) == st
         assert L.flce_backward(ctypes.byref(p), A, A, A, A, A, A, A, A, 1 << 40, None) == st
     p = flce.make_problem(64, 64, 512)
-    p.reserved1 = 1
+    p.dw_fp32 = 2
     assert L.flce_forward(ctypes.byref(p), A, A, A, A, A, A, 1 << 40, None) == 1
     # in-op label shift: T must divide BT and be >= 0
     for T in (-1, 48):
@@ -169,3 +169,124 @@ def test_kernel_code_hash_ignores_comments_only(tmp_path):
     assert bench.csrc_sha16(str(tmp_path)) == base
     f.write_text(text.replace("kStatusBadLabel = 5", "kStatusBadLabel = 6"))
     assert bench.csrc_sha16(str(tmp_path)) != base
+
+
+def test_row_stride_checks_before_any_launch():
+    """ldx/ldw/lddx/lddw: 0 means H; below H is invalid; a row pitch that is
+    not a whole number of 16-byte units is misaligned; both found on the
+    host."""
+    import ctypes
+    L = binding.lib()
+    ok = flce.make_problem(64, 64, 512, ldx=72, ldw=128, lddx=64, lddw=96)
+    assert flce.flce_workspace_size(ok, flce.FLCE_OP_FUSED) > 0
+    # strides do not change the workspace
+    assert (flce.flce_workspace_size(ok, flce.FLCE_OP_FUSED)
+            == flce.flce_workspace_size(flce.make_problem(64, 64, 512), flce.FLCE_OP_FUSED))
+    for field in ("ldx", "ldw", "lddx", "lddw"):
+        for value, st in [(56, 1), (-8, 1), (68, 3), (1 << 31, 2)]:
+            p = flce.make_problem(64, 64, 512, **{field: value})
+            assert flce.flce_workspace_size(p, flce.FLCE_OP_FUSED) == 0
+            assert L.flce_fused(ctypes.byref(p), A, A, A, 1.0, A, A, A, A, 1 << 40, None) == st
+    # fp32 rows: a stride of 68 elements is 272 bytes, a whole number of 16-byte units
+    p = flce.make_problem(64, 64, 512, dtype=flce.FLCE_FP32, ldx=68)
+    assert flce.flce_workspace_size(p, flce.FLCE_OP_FUSED) > 0
+
+
+def test_ce_host_checks():
+    import ctypes
+    L = binding.lib()
+    mk = flce.make_ce_problem
+    p = mk(1000, 50257)
+    fwd = flce.flce_ce_workspace_size(p, flce.FLCE_OP_FORWARD)
+    bwd = flce.flce_ce_workspace_size(p, flce.FLCE_OP_BACKWARD)
+    assert fwd >= 256 + 4 * 1000 and bwd == 256
+    assert flce.flce_ce_workspace_size(p, flce.FLCE_OP_FUSED) == 0
+    sh = mk(1000, 50257, shift_seq_len=100)
+    assert flce.flce_ce_workspace_size(sh, flce.FLCE_OP_BACKWARD) == 256 + 8192  # 256-aligned
+    for bad, st in [(mk(-1, 10), 1), (mk(4, 0), 1), (mk(4, 10, ld=9), 1), (mk(4, 10, ld_grad=3), 1),
+                    (mk(4, 10, dtype=5), 2), (mk(4, 1 << 31), 2), (mk(6, 10, shift_seq_len=4), 1)]:
+        assert flce.flce_ce_workspace_size(bad, flce.FLCE_OP_FORWARD) == 0
+        assert L.flce_ce_forward(ctypes.byref(bad), A, A, A, A, A, 1 << 40, None) == st
+        assert L.flce_ce_backward(ctypes.byref(bad), A, A, A, A, A, A, 1 << 40, None) == st
+    ok = mk(4, 10)
+    # bf16 logits need 2-byte alignment only (rows of odd V are fine), fp32 4
+    assert L.flce_ce_forward(ctypes.byref(ok), A + 1, A, A, A, A, 1 << 40, None) == 3
+    assert L.flce_ce_forward(ctypes.byref(mk(4, 10, dtype=flce.FLCE_FP32)), A + 2, A, A, A, A,
+                             1 << 40, None) == 3
+    assert L.flce_ce_forward(ctypes.byref(ok), A, A + 4, A, A, A, 1 << 40, None) == 3
+    assert L.flce_ce_forward(ctypes.byref(ok), A, A, A, A, A + 8, 1 << 40, None) == 3
+    assert L.flce_ce_forward(ctypes.byref(ok), A, A, A, A, A, 10, None) == 4
+    assert L.flce_ce_forward(ctypes.byref(ok), A, A, 0, A, A, 1 << 40, None) == 1
+    assert L.flce_ce_backward(ctypes.byref(ok), A, A, A, 0, A, A, 1 << 40, None) == 1
+    assert L.flce_ce_backward(ctypes.byref(ok), A, A, A, A, A + 1, A, 1 << 40, None) == 3
+
+
+def test_binding_checks_tensors_against_the_problem():
+    """The binding raises before taking a pointer when a tensor's layout,
+    dtype or device differs from what the problem says (no GPU needed:
+    every case fails a check first)."""
+    import torch
+    X = torch.zeros(8, 64, dtype=torch.bfloat16)
+    W = torch.zeros(40, 64, dtype=torch.bfloat16)
+    lab = torch.zeros(8, dtype=torch.int64)
+    with pytest.raises(ValueError, match="CUDA"):
+        flce.fused(X, W, lab)                       # host tensors never reach a kernel
+    with pytest.raises(ValueError, match="unit-stride"):
+        binding._problem_of(torch.zeros(64, 8, dtype=torch.bfloat16).t(), W, -100, 0.0)
+    with pytest.raises(ValueError, match="both"):
+        binding._problem_of(X, W.float(), -100, 0.0)
+    wide = torch.zeros(8, 96, dtype=torch.bfloat16)
+    p = binding._problem_of(wide[:, 16:80], W, -100, 0.0)
+    assert (p.ldx, p.ldw, p.H) == (96, 64, 64)      # a column slice: row stride 96
+    p = flce.make_problem(8, 64, 40)
+    for kw, msg in [(dict(X=X[:, :32]), "shape"), (dict(labels=lab.int()), "int64"),
+                    (dict(X=wide[:, :64]), "row stride 96, the problem says 64"),
+                    (dict(X=X), "CUDA")]:
+        with pytest.raises(ValueError, match=msg):
+            binding._check_flce(p, **kw)
+    with pytest.raises(ValueError, match="CUDA"):
+        flce.ce_forward(torch.zeros(4, 10), torch.zeros(4, dtype=torch.int64))
+
+
+@pytest.mark.parametrize("name", ["gpt2_small", "llama3_8b", "gemma2_softcap"])
+def test_workspace_below_one_logits_tensor_when_capped_or_fp32_dW(name):
+    """The survey's bound on peak extra HBM, below one bf16 BT x V tensor,
+    holds in two modes: under a workspace cap of exactly that size (the
+    automatic schedule then gives up the fused-in-forward plan, or narrows
+    the recompute chunk, as needed), and with an fp32 dW, where the
+    fused-in-forward schedule keeps its running sum in dW itself."""
+    w = inputs.WORKLOADS[name]
+    logits_bytes = 2 * w.BT * w.V
+    p = flce.make_problem(w.BT, w.H, w.V, flce.FLCE_BF16, softcap=w.softcap)
+    free = flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
+    prev = flce.flce_set_workspace_limit(logits_bytes)
+    try:
+        capped = flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
+        # a forced schedule ignores the cap
+        old = flce.flce_set_schedule(flce.FLCE_SCHEDULE_FUSED_FORWARD)
+        forced = flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
+        flce.flce_set_schedule(old)
+        # a cap below every plan: the smallest recompute plan
+        flce.flce_set_workspace_limit(1)
+        smallest = flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
+    finally:
+        flce.flce_set_workspace_limit(prev)
+    assert capped < logits_bytes and (capped == free or capped < free)
+    assert forced == free and 0 < smallest <= capped
+    p32 = flce.make_problem(w.BT, w.H, w.V, flce.FLCE_BF16, softcap=w.softcap, dw_fp32=1)
+    f32 = flce.flce_workspace_size(p32, flce.FLCE_OP_FUSED)
+    assert f32 < logits_bytes
+    assert free - f32 == -(-w.V * w.H * 4 // 256) * 256     # exactly the fp32 sum
+
+
+def test_dw_fp32_problem_checks():
+    import ctypes
+    L = binding.lib()
+    # fp32 dW rows: a stride of 68 floats is 272 bytes (16-byte multiple); as
+    # bf16 it would be 136 bytes (not)
+    assert flce.flce_workspace_size(flce.make_problem(64, 64, 512, lddw=68, dw_fp32=1), 2) > 0
+    p = flce.make_problem(64, 64, 512, lddw=68)
+    assert L.flce_fused(ctypes.byref(p), A, A, A, 1.0, A, A, A, A, 1 << 40, None) == 3
+    for bad in (-1, 2):
+        p = flce.make_problem(64, 64, 512, dw_fp32=bad)
+        assert L.flce_fused(ctypes.byref(p), A, A, A, 1.0, A, A, A, A, 1 << 40, None) == 1

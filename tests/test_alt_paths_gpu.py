@@ -4,7 +4,9 @@ environment variable, run in a child process against the oracle:
   FLCE_CTA_PAIR=0  single-CTA 128 x 256 tcgen05 tiles (four epilogue warps,
                    one LSE partial per 256 columns) instead of CTA pairs.
 
-The child prints one JSON line of errors; the parent checks the tolerances.
+The child prints one JSON line of errors; the parent checks the tolerances,
+and that row-strided views (X a column slice, dX and dW slices of wider
+buffers) give the dense results bit for bit on this path too.
 """
 import json
 import os
@@ -35,15 +37,37 @@ for (BT, H, V, cap, ign, seed) in %(cases)r:
         loss, dX, dW = flce.fused(X.to(dev), W.to(dev), lab.to(dev), softcap=cap, dloss=0.5)
         flce.flce_set_schedule(prev)
         torch.cuda.synchronize()
+        # the same call on row-strided views: X a column slice, dX and dW
+        # written into slices of wider buffers (the epilogues' own stores)
+        prev = flce.flce_set_schedule(sched)
+        xb = torch.zeros(BT, H + 16, dtype=torch.bfloat16, device=dev)
+        xb[:, :H] = X.to(dev)
+        gx = torch.full((BT, H + 8), 3.0, dtype=torch.bfloat16, device=dev)
+        gw = torch.full((V, H + 24), 3.0, dtype=torch.bfloat16, device=dev)
+        l2, dX2, dW2 = flce.fused(xb[:, :H], W.to(dev), lab.to(dev), softcap=cap, dloss=0.5,
+                                  dX=gx[:, :H], dW=gw[:, :H])
+        flce.flce_set_schedule(prev)
+        torch.cuda.synchronize()
+        # and an fp32 dW (the epilogues' fp32 stores), equal to dW once rounded
+        prev = flce.flce_set_schedule(sched)
+        l3, dX3, dW3 = flce.fused(X.to(dev), W.to(dev), lab.to(dev), softcap=cap, dloss=0.5,
+                                  dw_fp32=True)
+        flce.flce_set_schedule(prev)
+        torch.cuda.synchronize()
+        same = (l2.item() == loss.item() and torch.equal(dX2, dX) and torch.equal(dW2, dW)
+                and bool((gx[:, H:] == 3.0).all()) and bool((gw[:, H:] == 3.0).all())
+                and torch.equal(dW3.to(torch.bfloat16), dW) and torch.equal(dX3, dX))
         out.append(dict(case=[BT, H, V], sched=sched,
                         loss=rel_scalar(loss.item(), o["loss"]),
-                        dX=rel_fro(to_np(dX), o["dX"]), dW=rel_fro(to_np(dW), o["dW"])))
+                        dX=rel_fro(to_np(dX), o["dX"]), dW=rel_fro(to_np(dW), o["dW"]),
+                        strided_same=same))
 print(json.dumps(out))
 """
 
 CASES = [
     (600, 192, 5000, 0.0, 0.10, 31),     # two row chunks, ragged V
     (520, 1096, 2100, 30.0, 0.05, 32),   # H > 1024, softcap
+    (200, 64, 40000, 0.0, 0.10, 33),     # recompute: two vocabulary chunks (dX running sum)
 ]
 
 
@@ -63,3 +87,4 @@ def test_alternative_path_matches_oracle(env, cuda_device):
         assert d["loss"] <= tol["loss"], d
         assert d["dX"] <= tol["grad"], d
         assert d["dW"] <= tol["grad"], d
+        assert d["strided_same"], d

@@ -135,3 +135,80 @@ def test_ragged_bt_sweep_rows(idx, cuda_device):
     o = run_oracle(X[Ri].cpu(), W.cpu(), labc[R], n_valid=nv, want_dW=False)
     assert rel_fro(to_np(dX[Ri]), o["dX"]) <= TOL["bf16"]["grad"]
     assert bool(torch.isfinite(dW).all())
+
+
+def _pairs_problem(w, D, seed, device):
+    """A full-size problem whose BT rows are D distinct (hidden state, label)
+    pairs, pair d repeated count_d times and scattered by a seeded
+    permutation over every row chunk.  Counts come in four classes of D/4
+    pairs with unequal multiplicities.  Returns the distinct pairs, the class
+    of each pair, the class counts and the row -> pair index."""
+    Xd, W, labd = inputs.make_workload(w, device=device, BT=D)
+    labd = labd.clone()
+    if w.ignore_frac > 0:
+        labd[[3, 22, 41]] = inputs.IGNORE_INDEX      # ignored pairs in three classes
+    base = w.BT // D
+    counts = [base * 4 // 10, base * 7 // 10, base * 12 // 10]
+    counts.append(4 * base - sum(counts))            # the classes together fill BT
+    per_class = D // 4
+    cls = np.repeat(np.arange(4), per_class)
+    mult = np.array([counts[c] for c in cls])
+    assert mult.sum() == w.BT and len(set(counts)) == 4
+    g = torch.Generator().manual_seed(seed)
+    idx = torch.repeat_interleave(torch.arange(D), torch.tensor(mult))
+    idx = idx[torch.randperm(w.BT, generator=g)]
+    return Xd, W, labd, cls, counts, idx
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_dW_vs_oracle(name, cuda_device):
+    """The whole V x H dW and BT x H dX of a full-size call (automatic
+    schedule, the bench's launch configuration, every row chunk, the fp32
+    running sum read back) against the oracle element by element.  With the
+    rows built from D distinct pairs, dW = sum_d count_d G_d^T x_d: the oracle
+    runs each multiplicity class's pairs once (global N_valid) and the class
+    dW's are weighted by the class count, in fp64."""
+    w = inputs.WORKLOADS[name]
+    D = 64
+    Xd, W, labd, cls, counts, idx = _pairs_problem(w, D, seed=17, device=cuda_device)
+    idx_d = idx.to(cuda_device)
+    X = Xd[idx_d].contiguous()
+    lab = labd[idx_d].contiguous()
+    p = flce.make_problem(w.BT, w.H, w.V, X.dtype, softcap=w.softcap)
+    ws = flce.workspace(p, flce.FLCE_OP_FUSED, cuda_device)
+    loss, dX, dW = flce.fused(X, W, lab, softcap=w.softcap, ws=ws)
+    status, nv = flce.flce_get_device_status(ws)
+    labc = labd.cpu()
+    valid = (labc != inputs.IGNORE_INDEX).numpy()
+    n_global = int(sum(counts[c] for c, v in zip(cls, valid) if v))
+    assert status == 0 and nv == n_global == oracle.count_valid(lab.cpu().numpy())
+    del ws
+    Xc, Wc = Xd.cpu(), W.cpu()
+    dW_ref = None
+    dX_pairs = np.zeros((D, w.H))
+    loss_ref = 0.0
+    for c in range(4):
+        rows = np.nonzero(cls == c)[0]
+        o = run_oracle(Xc[rows], Wc, labc[rows], softcap=w.softcap, n_valid=n_global)
+        dX_pairs[rows] = o["dX"]
+        loss_ref += counts[c] * o["loss"]
+        o["dW"] *= counts[c]
+        if dW_ref is None:
+            dW_ref = o["dW"]
+        else:
+            dW_ref += o["dW"]
+        del o
+    tol = TOL["bf16"]
+    assert rel_scalar(loss.item(), loss_ref) <= tol["loss"]
+    # dX: every row against its pair's oracle row
+    dX_ref = torch.from_numpy(dX_pairs).to(cuda_device)[idx_d]
+    err = float((dX.double() - dX_ref).norm() / dX_ref.norm())
+    assert err <= tol["grad"], err
+    del dX_ref
+    # dW: the whole matrix, compared in row blocks on the GPU
+    num = den = 0.0
+    for r0 in range(0, w.V, 16384):
+        ref = torch.from_numpy(dW_ref[r0:r0 + 16384]).to(cuda_device)
+        num += float(((dW[r0:r0 + 16384].double() - ref) ** 2).sum())
+        den += float((ref ** 2).sum())
+    assert (num / den) ** 0.5 <= tol["grad"], (num / den) ** 0.5

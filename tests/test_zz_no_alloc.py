@@ -4,10 +4,13 @@ the GPU's memory, or a caller from another language that can only pass the
 tensors it was given).  It takes no workspace; its scratch space is a fixed
 64 MiB array inside the library, shared by every call on a device.
 
-The GPU test calls it twice in a row through the C ABI, on two different
-problems, and checks each result against flce_fused run with an ordinary
-workspace, with the tolerances of the other parity tests.  The file is named
-so that pytest collects it last.
+The GPU test calls it several times in a row through the C ABI, on problems
+of different shapes and both schedules (the fused-in-forward one keeps an
+fp32 dW running sum and dX split slabs in the array, the in-op label shift a
+copy of the labels), so every call runs on scratch a different call left
+behind.  Each result must equal flce_fused with an ordinary workspace bit
+for bit: the same kernels run in the same order on the same data.  The file
+is named so that pytest collects it last.
 """
 import ctypes
 
@@ -16,7 +19,6 @@ import torch
 
 import linear_cross_entropy_tiles_b200 as flce
 from linear_cross_entropy_tiles_b200 import binding, inputs
-from parity import TOL, rel_fro, rel_scalar
 
 
 def test_rejects_problems_beyond_the_scratch_size():
@@ -30,27 +32,28 @@ def test_rejects_problems_beyond_the_scratch_size():
     assert flce.flce_workspace_size(p, flce.FLCE_OP_FUSED) > 64 << 20
 
 
-def _call_pair(BT, H, V, softcap, seed, dev):
-    X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.05, 0.1, seed=seed, device=dev)
-    p = flce.make_problem(BT, H, V, X.dtype, softcap=softcap)
-    assert flce.flce_workspace_size(p, flce.FLCE_OP_FUSED) <= 64 << 20
-    # Reference: the existing entry point with its own workspace.
-    ref = flce.fused(X, W, lab, softcap=softcap, dloss=0.75)
-    # The allocation-free entry point, through the C ABI.
-    loss = torch.empty(1, dtype=torch.float32, device=dev)
-    dX, dW = torch.empty_like(X), torch.empty_like(W)
-    binding.flce_fused_noalloc(p, X, W, lab, 0.75, loss, dX, dW)
-    torch.cuda.synchronize()
-    return ref, (loss, dX, dW)
+# BT, H, V, softcap, shift_seq_len, seed: recompute (BT < 512) and
+# fused-in-forward (BT >= 512: two row chunks, fp32 dW sum, dX split slabs)
+CALLS = [(300, 192, 1000, 0.0, 0, 41),
+         (1024, 256, 4000, 0.0, 0, 43),
+         (200, 128, 3000, 30.0, 0, 42),
+         (1024, 128, 2000, 10.0, 256, 44),
+         (600, 192, 1000, 0.0, 0, 45)]
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_fused_on_two_calls_in_a_row(cuda_device):
-    tol = TOL["bf16"]
-    # Two different problems back to back: the second call runs on scratch
-    # the first one left behind.
-    for BT, H, V, cap, seed in [(300, 192, 1000, 0.0, 41), (200, 128, 3000, 30.0, 42)]:
-        (l0, dx0, dw0), (l1, dx1, dw1) = _call_pair(BT, H, V, cap, seed, cuda_device)
-        assert rel_scalar(l1.item(), l0.item()) <= tol["loss"]
-        assert rel_fro(dx1.float().cpu().numpy(), dx0.float().cpu().numpy()) <= tol["grad"]
-        assert rel_fro(dw1.float().cpu().numpy(), dw0.float().cpu().numpy()) <= tol["grad"]
+def test_noalloc_equals_fused_bitwise_on_calls_in_a_row(cuda_device):
+    for BT, H, V, cap, T, seed in CALLS:
+        X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.05, 0.1, seed=seed,
+                                       device=cuda_device)
+        p = flce.make_problem(BT, H, V, X.dtype, softcap=cap, shift_seq_len=T)
+        assert 0 < flce.flce_workspace_size(p, flce.FLCE_OP_FUSED) <= 64 << 20
+        # Reference: the existing entry point with its own workspace.
+        ref = flce.fused(X, W, lab, softcap=cap, dloss=0.75, shift_seq_len=T)
+        # The allocation-free entry point, through the C ABI.
+        loss = torch.empty(1, dtype=torch.float32, device=cuda_device)
+        dX, dW = torch.empty_like(X), torch.empty_like(W)
+        binding.flce_fused_noalloc(p, X, W, lab, 0.75, loss, dX, dW)
+        torch.cuda.synchronize()
+        assert loss.item() == ref[0].item(), (BT, H, V)
+        assert torch.equal(dX, ref[1]) and torch.equal(dW, ref[2]), (BT, H, V)
