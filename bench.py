@@ -4,15 +4,16 @@
 
 One step = one flce_fused call over one batch of synthetic inputs already
 resident in HBM: labels check, then per row chunk the forward GEMM (logits,
-online max / sum-exp, q stored in bf16), the in-place G pass, the dX GEMM
-and the accumulating dW GEMM, then the loss (the fused-in-forward schedule;
+per-row sum-exp, q = exp(y - R) stored in bf16 against one reference per
+row), the per-row lse / scale / label-column pass, the dX GEMM (rows scaled
+by their factor) and the accumulating dW GEMM, then the loss (the fused-in-forward schedule;
 BT < 512 uses the two-pass recompute schedule).  Prints one JSON line.
 
 Multi-GPU: one process per GPU (torchrun), data parallel over rows (weak
 scaling: every rank holds BT rows of a global batch of N*BT rows and the same
 W).  Each timed step counts the rank's non-ignored labels, all-reduces that
-count (the divisor of the global mean), runs flce_fused_global, and
-all-reduces the loss shares and dW (bf16) over NCCL.  --parallel replicas
+count (the divisor of the global mean), runs flce_fused_global (dW written
+in fp32), and all-reduces the loss shares and the fp32 dW over NCCL.  --parallel replicas
 runs independent copies instead (no collective).  Time is the max over ranks
 of the device-timed region; value = tokens of all ranks / that time.
 
@@ -506,6 +507,8 @@ def main():
     ap.add_argument("--ragged-limit", type=int, default=0)
     ap.add_argument("--prof-steps", type=int, default=20,
                     help="steps of the second, per-launch-timed loop")
+    ap.add_argument("--dw-reduce", default="fp32", choices=["fp32", "bf16"],
+                    help="data parallel: dtype in which dW is written and summed over ranks")
     ap.add_argument("--parallel", default=None, choices=["dp", "replicas"],
                     help="with several ranks: data parallel over rows (default) or "
                          "independent replicas; 'dp' on one rank runs the same step "
@@ -552,15 +555,18 @@ def main():
     if args.parallel == "dp" and world > 1:
         W = inputs.make_workload(inputs.WORKLOADS[args.workload], device=dev, BT=1)[1]
     flce.flce_set_schedule({"auto": 0, "recompute": 1, "fused_fwd": 2}[args.schedule])
-    p = flce.make_problem(w.BT, w.H, w.V, X.dtype, softcap=w.softcap)
+    dp_mode = args.parallel == "dp"
+    # Data parallel: each rank writes its dW share in fp32 and the ranks sum
+    # it in fp32 (--dw-reduce bf16: bf16 shares summed in bf16).
+    dw32 = dp_mode and args.dw_reduce == "fp32" and w.dtype == "bf16"
+    p = flce.make_problem(w.BT, w.H, w.V, X.dtype, softcap=w.softcap, dw_fp32=int(dw32))
     torch.cuda.synchronize()
     ws = flce.workspace(p, flce.FLCE_OP_FUSED, dev)
     loss = torch.empty(1, dtype=torch.float32, device=dev)
     dX = torch.empty_like(X)
-    dW = torch.empty_like(W)
+    dW = torch.empty(W.shape, dtype=torch.float32 if dw32 else W.dtype, device=dev)
     stream = torch.cuda.current_stream()
 
-    dp_mode = args.parallel == "dp"
     n_valid_buf = torch.empty(1, dtype=torch.int64, device=dev)
 
     def compute():
@@ -603,7 +609,7 @@ def main():
     # G GEMMs recompute the logits X W^T, the dX / dW GEMMs are G W and G^T X).
     gemm_flops = 2.0 * w.BT * w.H * w.V
     flops_per_step = {k: gemm_flops for k in ("lse_gemm", "grad_gemm", "dx_gemm", "dw_gemm",
-                                              "lse_p_gemm", "dw_acc_gemm", "simt_lse",
+                                              "lse_q_gemm", "dw_acc_gemm", "simt_lse",
                                               "simt_grad", "simt_dx", "simt_dw")}
     dom_time_per_step = by_kind[dom][0] / prof_steps
     launches_dom = by_kind[dom][1] / prof_steps

@@ -131,138 +131,141 @@ __global__ void finalize_kernel(const float* __restrict__ row_loss, int64_t BT,
   }
 }
 
-// Fused-in-forward schedule, one block (256 threads) per row of a row chunk:
-// fold the row's (reference, sum) partials into lse in a fixed order,
-// write lse and the row's NLL, then turn the row's q = exp(y - reference) *
-// dy/dz (bf16, written by the forward GEMM) into G in place:
-//   G_ij = q_ij * exp(reference - lse) * dloss / N              (j != label)
-//   G_il = (exp(y_il - lse) - 1) * dy/dz * dloss / N            (label column,
-//          from the fp32 target logit, so p close to 1 loses nothing)
-// with dy/dz = 1 - (y/c)^2 under a softcap c, 1 otherwise.  Ignored rows
-// become zero.
-constexpr int kLseGradThreads = 256;
+// Fused-in-forward schedule, after a row chunk's forward GEMM.  Every row's
+// partials -- per vocabulary slice the largest u = y log2(e) and the sum of
+// exp2(u - R) -- share the row's one reference R (0, or the row's maximum
+// after a recomputation), so for each row of the chunk:
+//   S = sum over slices of the sums (in slice order), lse = (R + log2 S) ln 2,
+//   the row's NLL, f = exp2(R - log2 S - R) = 1 / S (0 for an ignored row),
+//   row_scale = f dloss / N (the dX epilogue's factor),
+//   Xs = bf16(f x) (the dW GEMM's operand), and the label column of the
+//   chunk buffer replaced by (p - 1) dy/dz / f -- G / (f dloss / N) there,
+//   computed from the fp32 target logit so a probability near 1 loses
+//   nothing -- after which G = (dloss / N) diag(f) Q everywhere.
+// q, f and Xs stay inside bf16's normal range while the row's largest u lies
+// in [-kRefWindow, kRefWindow]; a valid row outside it (or with a sum that is
+// not finite) is left by pass 1, which records its exact maximum as its new
+// reference and flags its 32-row group (every other row keeps reference 0).
+// The forward GEMM then recomputes the flagged groups against those
+// references -- rewriting their rows of P whole, label columns included --
+// and pass 2 finishes every row of the flagged groups (blocks of unflagged
+// groups return at once); a row that was fine gets the same values again.
+constexpr int kLseQRows = 32;       // rows per block: one flag group
+constexpr int kLseQThreads = 256;   // eight warps; lane = row of the group
+constexpr float kRefWindow = 64.f;  // log2 units
 
-__global__ void __launch_bounds__(kLseGradThreads)
-    lse_grad_kernel(const float2* __restrict__ partial, int n_tiles, int part_shift, int64_t BT,
-                    int64_t row0,
-                    const float* __restrict__ target, const int64_t* __restrict__ labels,
-                    int64_t ignore_index, int64_t ncols, __nv_bfloat16* __restrict__ P,
-                    int64_t ldp, float* __restrict__ lse_out, float* __restrict__ row_loss,
-                    const WsHeader* hdr, float dloss, float softcap) {
-  __shared__ float red[kLseGradThreads / 32];
-  __shared__ float bcast;
+__global__ void __launch_bounds__(kLseQThreads)
+    lse_q_kernel(int pass, const float2* __restrict__ partial, int n_parts, int64_t BT,
+                 int64_t row0, int64_t rows, const float* __restrict__ target,
+                 const int64_t* __restrict__ labels, int64_t ignore_index,
+                 __nv_bfloat16* __restrict__ P, int64_t ldp, const __nv_bfloat16* __restrict__ X,
+                 int64_t ldx, int64_t H, __nv_bfloat16* __restrict__ Xs, float* __restrict__ ref,
+                 int* __restrict__ group_flags,
+                 float* __restrict__ lse_out, float* __restrict__ row_loss,
+                 float* __restrict__ row_scale, const WsHeader* hdr, float dloss,
+                 float softcap) {
+  __shared__ float s_max[kLseQThreads / 32][kLseQRows];
+  __shared__ float s_sum[kLseQThreads / 32][kLseQRows];
+  __shared__ float s_f[kLseQRows];
+  __shared__ int s_do[kLseQRows];  // this pass finishes the row
   if (hdr->status != 0) return;
-  const int64_t lrow = blockIdx.x;
-  const int64_t row = row0 + lrow;
+  const int group = blockIdx.x;
+  if (pass == 2 && group_flags[group] == 0) return;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  const float2* pr = partial + row;
-  // ---- lse: max over tiles, then sum of s_t * exp2(m_t - max) ----
-  float m = -INFINITY;
-  for (int t = tid; t < n_tiles; t += kLseGradThreads) m = fmaxf(m, pr[size_t(t) * BT].x);
+  const int64_t lrow = int64_t(group) * kLseQRows + lane;
+  const bool in = lrow < rows;
+  const int64_t row = row0 + lrow;
+  // ---- per row: max and sum of the partials; warp w takes slices w, w+8, ...
+  float m = -INFINITY, sum = 0.f;
+  if (in) {
+    const float2* pr = partial + row;
+    for (int t = wid; t < n_parts; t += 4 * (kLseQThreads / 32)) {
+      float2 v[4];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  if (lane == 0) red[wid] = m;
-  __syncthreads();
-  if (tid == 0) {
-    float mm = red[0];
-    for (int w = 1; w < kLseGradThreads / 32; ++w) mm = fmaxf(mm, red[w]);
-    bcast = mm;
-  }
-  __syncthreads();
-  m = bcast;
-  float s = 0.f;
-  for (int t = tid; t < n_tiles; t += kLseGradThreads) {
-    const float2 q = pr[size_t(t) * BT];
-    s += q.y * exp2f(q.x - m);
-  }
+      for (int u = 0; u < 4; ++u) {
+        const int tt = t + u * (kLseQThreads / 32);
+        v[u] = tt < n_parts ? pr[size_t(tt) * BT] : make_float2(-INFINITY, 0.f);
+      }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  __syncthreads();
-  if (lane == 0) red[wid] = s;
-  __syncthreads();
-  if (tid == 0) {
-    float ss = 0.f;
-    for (int w = 0; w < kLseGradThreads / 32; ++w) ss += red[w];
-    bcast = m + log2f(ss);
-  }
-  __syncthreads();
-  const float lse2 = bcast;  // lse in base-2 units
-  const int64_t lab = labels[row];
-  const bool valid = lab != ignore_index;
-  const long long nv = hdr->n_valid;
-  const float scale = (valid && nv > 0) ? dloss / float(nv) : 0.f;
-  const bool cap = softcap > 0.f;
-  const float inv_c = cap ? 1.f / softcap : 0.f;
-  const float tgt = valid ? target[row] : 0.f;
-  if (tid == 0) {
-    const float l = lse2 * 0.69314718055994531f;
-    lse_out[row] = l;
-    row_loss[row] = valid ? l - tgt : 0.f;
-  }
-  // ---- G in place, 8 columns (16 bytes) per thread per step, four steps'
-  // loads in flight at a time ----
-  __nv_bfloat16* prow = P + lrow * ldp;
-  constexpr int kUnroll = 4;
-  const int64_t stride = int64_t(kLseGradThreads) * 8;
-  if (scale == 0.f) {  // ignored row (or no valid row at all): G is zero
-    for (int64_t j0 = int64_t(tid) * 8; j0 < ncols; j0 += stride)
-      *reinterpret_cast<uint4*>(prow + j0) = make_uint4(0u, 0u, 0u, 0u);
-    return;
-  }
-  float glab;  // G at the label column, from the fp32 target logit
-  {
-    float d = 1.f;
-    if (cap) {
-      const float t = tgt * inv_c;
-      d = 1.f - t * t;
-    }
-    glab = (exp2f(fmaf(tgt, 1.4426950408889634f, -lse2)) - 1.f) * d * scale;
-  }
-  for (int64_t j0 = int64_t(tid) * 8; j0 < ncols; j0 += kUnroll * stride) {
-    uint4 raw[kUnroll];
-    float f[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = j0 + u * stride;
-      if (j < ncols) {
-        raw[u] = *reinterpret_cast<const uint4*>(prow + j);
-        f[u] = pr[size_t(j >> part_shift) * BT].x;  // the column's partial slice max
+      for (int u = 0; u < 4; ++u) {
+        m = fmaxf(m, v[u].x);
+        sum += v[u].y;
       }
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = j0 + u * stride;
-      if (j >= ncols) break;
-      const float fu = exp2f(f[u] - lse2) * scale;
-      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw[u]);
-      const int64_t rel = lab - j;
-      if (rel >= 0 && rel < 8) {  // the label column is in this piece
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 pv = __bfloat1622float2(h[q]);
-          const float g0 = (2 * q == rel) ? glab : pv.x * fu;
-          const float g1 = (2 * q + 1 == rel) ? glab : pv.y * fu;
-          h[q] = __floats2bfloat162_rn(g0, g1);
-        }
+  }
+  s_max[wid][lane] = m;
+  s_sum[wid][lane] = sum;
+  __syncthreads();
+  if (wid == 0) {
+    float M = s_max[0][lane], S = s_sum[0][lane];
+    for (int w = 1; w < kLseQThreads / 32; ++w) {
+      M = fmaxf(M, s_max[w][lane]);
+      S += s_sum[w][lane];
+    }
+    const int64_t lab = in ? labels[row] : ignore_index;
+    const bool keep = lab != ignore_index;
+    bool finish = in;
+    float f = 0.f;
+    if (finish) {
+      const float R = pass == 1 ? 0.f : ref[lrow];
+      const bool ok = M >= -kRefWindow && M <= kRefWindow && S < INFINITY;
+      if (pass == 1 && keep && !ok) {
+        ref[lrow] = M;  // recompute against the row's exact maximum
+        finish = false;
       } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 pv = __bfloat1622float2(h[q]);
-          h[q] = __floats2bfloat162_rn(pv.x * fu, pv.y * fu);
+        if (pass == 1) ref[lrow] = 0.f;
+        const float lse2 = R + log2f(S);
+        const float l = lse2 * 0.69314718055994531f;
+        lse_out[row] = l;
+        const float tgt = keep ? target[row] : 0.f;
+        row_loss[row] = keep ? l - tgt : 0.f;
+        const long long nv = hdr->n_valid;
+        f = keep ? 1.f / S : 0.f;
+        row_scale[lrow] = keep && nv > 0 ? f * (dloss / float(nv)) : 0.f;
+        if (keep) {
+          float d = 1.f;
+          if (softcap > 0.f) {
+            const float t = tgt / softcap;
+            d = 1.f - t * t;
+          }
+          const float p = exp2f(fmaf(tgt, 1.4426950408889634f, -lse2));
+          P[lrow * ldp + lab] = __float2bfloat16_rn((p - 1.f) * d * S);
         }
       }
-      *reinterpret_cast<uint4*>(prow + j) = raw[u];
     }
+    s_do[lane] = finish ? 1 : 0;
+    s_f[lane] = f;
+    const unsigned any = __ballot_sync(0xffffffffu, pass == 1 && in && keep && !finish);
+    if (pass == 1 && lane == 0) group_flags[group] = any != 0u;
+  }
+  __syncthreads();
+  // ---- Xs = bf16(f x) for the rows this pass finished: 8 columns per thread
+  const int64_t vecs = H / 8;
+  for (int64_t e = tid; e < int64_t(kLseQRows) * vecs; e += kLseQThreads) {
+    const int rr = int(e / vecs);
+    const int64_t k = (e - int64_t(rr) * vecs) * 8;
+    if (!s_do[rr]) continue;
+    const int64_t lr = int64_t(group) * kLseQRows + rr;
+    const float f = s_f[rr];
+    uint4 raw = *reinterpret_cast<const uint4*>(X + (row0 + lr) * ldx + k);
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 v = __bfloat1622float2(h[q]);
+      h[q] = __floats2bfloat162_rn(v.x * f, v.y * f);
+    }
+    *reinterpret_cast<uint4*>(Xs + lr * H + k) = raw;
   }
 }
 
-// dX rows of a row chunk from its K-split slabs: out = bf16(sum_s slab_s),
-// summed in split order.  The slabs are dense rows of H; output rows are
-// ld_out apart.  n (rows * H) and H are multiples of 8, as is ld_out.
+// dX rows of a row chunk from its K-split slabs: out = bf16(sum_s slab_s *
+// row_scale[row]), summed in split order (row_scale null: 1).  The slabs are
+// dense rows of H; output rows are ld_out apart.  n (rows * H) and H are
+// multiples of 8, as is ld_out.
 __global__ void slab_reduce_kernel(const float* __restrict__ slabs, int n_slabs,
                                    int64_t slab_stride, int64_t n, int64_t H,
                                    __nv_bfloat16* __restrict__ out, int64_t ld_out,
-                                   const WsHeader* hdr) {
+                                   const float* __restrict__ row_scale, const WsHeader* hdr) {
   if (hdr->status != 0) return;
   for (int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 8; i < n;
        i += int64_t(gridDim.x) * blockDim.x * 8) {
@@ -275,8 +278,11 @@ __global__ void slab_reduce_kernel(const float* __restrict__ slabs, int n_slabs,
       a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
       b.x += d.x; b.y += d.y; b.z += d.z; b.w += d.w;
     }
-    __nv_bfloat162 h[4] = {__floats2bfloat162_rn(a.x, a.y), __floats2bfloat162_rn(a.z, a.w),
-                           __floats2bfloat162_rn(b.x, b.y), __floats2bfloat162_rn(b.z, b.w)};
+    const float f = row_scale ? row_scale[i / H] : 1.f;
+    __nv_bfloat162 h[4] = {__floats2bfloat162_rn(a.x * f, a.y * f),
+                           __floats2bfloat162_rn(a.z * f, a.w * f),
+                           __floats2bfloat162_rn(b.x * f, b.y * f),
+                           __floats2bfloat162_rn(b.z * f, b.w * f)};
     *reinterpret_cast<uint4*>(out + (i / H) * ld_out + i % H) = *reinterpret_cast<uint4*>(h);
   }
 }

@@ -50,6 +50,15 @@ struct CeElem<__nv_bfloat16> {
     (&v.x)[k >> 1] = pack_bf16x2(lo, hi);
   }
   __device__ static void store_one(__nv_bfloat16* p, float x) { *p = __float2bfloat16_rn(x); }
+  // Largest of the 8 values, compared as packed bf16 pairs.
+  __device__ static float vmax(const uint4& v) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const __nv_bfloat162 a = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+    return fmaxf(__low2float(a), __high2float(a));
+  }
+  __device__ static uint4 neg_inf() {  // 8 x bf16 -inf
+    return make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  }
 };
 template <>
 struct CeElem<float> {
@@ -61,6 +70,14 @@ struct CeElem<float> {
     (&v.x)[k + 1] = __float_as_uint(hi);
   }
   __device__ static void store_one(float* p, float x) { *p = x; }
+  __device__ static float vmax(const uint4& v) {
+    return fmaxf(fmaxf(__uint_as_float(v.x), __uint_as_float(v.y)),
+                 fmaxf(__uint_as_float(v.z), __uint_as_float(v.w)));
+  }
+  __device__ static uint4 neg_inf() {
+    const uint32_t n = 0xff800000u;
+    return make_uint4(n, n, n, n);
+  }
 };
 
 // Elements of a row before its first 16-byte boundary (at most V).
@@ -119,26 +136,26 @@ __global__ void __launch_bounds__(kCeThreads)
       const int64_t v = v0 + int64_t(u) * kCeThreads;
       if (v < nvec) raw[u] = __ldcs(zv + v);
     }
-    float uu[kCeUnroll][VE];
-    float gmax = -INFINITY;
+    // The group's largest logit (the softcap is increasing, so it caps the
+    // largest raw value); bf16 pairs compare packed.  Vectors past the row
+    // were not loaded: -inf.
+    float gz = -INFINITY;
 #pragma unroll
     for (int u = 0; u < kCeUnroll; ++u) {
-      const bool ok = v0 + int64_t(u) * kCeThreads < nvec;
-#pragma unroll
-      for (int k = 0; k < VE; ++k) {
-        uu[u][k] = ok ? ce_u<CAP>(E::get(raw[u], k), sc, inv_sc) : -INFINITY;
-        gmax = fmaxf(gmax, uu[u][k]);
-      }
+      if (v0 + int64_t(u) * kCeThreads >= nvec) raw[u] = E::neg_inf();
+      gz = fmaxf(gz, E::vmax(raw[u]));
     }
-    if (gmax == -INFINITY) continue;
-    const float mn = fmaxf(m, gmax);
+    if (gz == -INFINITY) continue;
+    const float mn = fmaxf(m, ce_u<CAP>(gz, sc, inv_sc));
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
     for (int u = 0; u < kCeUnroll; ++u) {
+      if (v0 + int64_t(u) * kCeThreads >= nvec) break;  // not loaded (a capped -inf is not 0)
 #pragma unroll
       for (int k = 0; k < VE; k += 2) {
-        a0 += ex2a(uu[u][k] - mn);
-        a1 += ex2a(uu[u][k + 1] - mn);
+        float d;
+        a0 += ex2a(fmaf(capped<CAP>(E::get(raw[u], k), sc, inv_sc, &d), kLog2e, -mn));
+        a1 += ex2a(fmaf(capped<CAP>(E::get(raw[u], k + 1), sc, inv_sc, &d), kLog2e, -mn));
       }
     }
     s = s * ex2a(m - mn) + (a0 + a1);

@@ -41,10 +41,11 @@ thread_local int32_t t_launches = 0;
 // Kernel kinds, in the order flce_kernel_name() names them.
 enum Kind : int32_t {
   K_LABELS = 0, K_LSE_GEMM, K_COMBINE, K_FINALIZE, K_GRAD_GEMM, K_DX_GEMM, K_DW_GEMM,
-  K_SIMT_LOGITS, K_SIMT_GRAD, K_SIMT_DX, K_SIMT_DW, K_MEMSET, K_LSEP_GEMM, K_LSE_GRAD,
+  K_SIMT_LOGITS, K_SIMT_GRAD, K_SIMT_DX, K_SIMT_DW, K_MEMSET, K_LSEQ_GEMM, K_LSEQ,
   K_DWACC_GEMM, K_DX_REDUCE, K_COUNT_VALID, K_SET_NVALID, K_SHIFT_LABELS,
   // launched from flce_ce.cu (kinds fixed in internal.h)
-  K_CE_FORWARD, K_CE_BACKWARD, K_CE_FUSED, K_NUM_KINDS
+  K_CE_FORWARD, K_CE_BACKWARD, K_CE_FUSED,
+  K_LSEQ_REPAIR, K_NUM_KINDS
 };
 static_assert(int32_t(K_CE_FORWARD) == int32_t(flce_internal::kKindCeForward) &&
                   int32_t(K_CE_BACKWARD) == int32_t(flce_internal::kKindCeBackward) &&
@@ -52,9 +53,9 @@ static_assert(int32_t(K_CE_FORWARD) == int32_t(flce_internal::kKindCeForward) &&
               "kernel kinds shared with flce_ce.cu");
 const char* const kKindNames[K_NUM_KINDS] = {
     "labels", "lse_gemm", "lse_combine", "loss_finalize", "grad_gemm", "dx_gemm", "dw_gemm",
-    "simt_lse", "simt_grad", "simt_dx", "simt_dw", "memset", "lse_p_gemm", "lse_grad",
+    "simt_lse", "simt_grad", "simt_dx", "simt_dw", "memset", "lse_q_gemm", "lse_q",
     "dw_acc_gemm", "dx_reduce", "count_valid", "set_n_valid", "shift_labels", "ce_forward",
-    "ce_backward", "ce_fused"};
+    "ce_backward", "ce_fused", "lse_q_repair_gemm"};
 
 // flce_fused schedule: 0 = choose, 1 = two-pass recompute, 2 = fused-in-forward.
 std::atomic<int32_t> g_schedule{0};
@@ -111,6 +112,9 @@ struct Plan {
   int64_t Cb = 0, n_row_chunks = 0, ldp = 0;
   int dx_splits = 1;      // K (vocabulary) splits of the chunk's dX GEMM
   size_t off_p = 0, off_dwacc = 0, off_dxslab = 0;
+  // per chunk row: prescaled X rows [Cb][H] bf16, exponent reference and dX
+  // factor; one recomputation flag per 32-row group
+  size_t off_xs = 0, off_ref = 0, off_rowscale = 0, off_flags = 0;
 };
 
 bool softcap_on(float c) { return c > 0.f && std::isfinite(c); }
@@ -241,6 +245,15 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl) {
     pl->off_dxslab = off;
     off = align256(off + size_t(pl->dx_splits) * size_t(pl->Cb) * size_t(H) * 4);
   }
+  const size_t cb = size_t(pl->Cb);
+  pl->off_xs = off;
+  off = align256(off + cb * size_t(H) * 2);
+  pl->off_ref = off;
+  off = align256(off + cb * 4);
+  pl->off_rowscale = off;
+  off = align256(off + cb * 4);
+  pl->off_flags = off;
+  off = align256(off + size_t(cdiv(pl->Cb, kLseQRows)) * 4);
   pl->total = off;
 }
 
@@ -398,7 +411,7 @@ cudaError_t launch_tc(const CUtensorMap& a, const CUtensorMap& b, const TcShape&
   constexpr int32_t kind_default =
       (MODE == EPI_LSE || MODE == EPI_LSE_CAP) ? K_LSE_GEMM
       : (MODE == EPI_GRAD || MODE == EPI_GRAD_CAP) ? K_GRAD_GEMM
-      : MODE == EPI_DX ? K_DX_GEMM : MODE == EPI_DW ? K_DW_GEMM : K_LSEP_GEMM;
+      : MODE == EPI_DX ? K_DX_GEMM : MODE == EPI_DW ? K_DW_GEMM : K_LSEQ_GEMM;
   const int32_t kind = kind_override >= 0 ? kind_override : kind_default;
   constexpr int STAGES = kStagesBN256;
   auto kern = tc_gemm_kernel<BN, A_MN, B_MN, MODE, STAGES>;
@@ -475,7 +488,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
   constexpr int32_t kind_default =
       (MODE == EPI_LSE || MODE == EPI_LSE_CAP) ? K_LSE_GEMM
       : (MODE == EPI_GRAD || MODE == EPI_GRAD_CAP) ? K_GRAD_GEMM
-      : MODE == EPI_DX ? K_DX_GEMM : MODE == EPI_DW ? K_DW_GEMM : K_LSEP_GEMM;
+      : MODE == EPI_DX ? K_DX_GEMM : MODE == EPI_DW ? K_DW_GEMM : K_LSEQ_GEMM;
   if (kind < 0) kind = kind_default;
   const bool pair = use_pair();
   TcShape sh = make_shape(g.M, g.N, g.K, 256, g.m_fast, pair ? kPairBM : kBM);
@@ -753,14 +766,23 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
 
 // flce_fused, fused-in-forward schedule (6*BT*H*V FLOP: no logit recompute).
 // For each chunk of Cb rows:
-//   lse_p GEMM   X_b W^T; epilogue stores p = exp(y - m) (bf16) into P, m a
-//                per-(row, slice) reference, the (m, sum) partials and the
-//                target logit
-//   lse_grad     lse and NLL of the chunk's rows; P becomes G in place
-//   dX GEMM      dX_b = G_b W        (K = all of V: complete, bf16 out)
-//   dW GEMM      dW  (+)= G_b^T X_b  (fp32 running sum over chunks, bf16 on
-//                the last chunk)
-// then the loss over all rows.  Labels were checked by the caller.
+//   lse_q GEMM   X_b W^T; epilogue stores q = exp(y - R) dy/dz (bf16) into P
+//                with one reference R per row (0), the (max, sum) partials
+//                and the target logit
+//   lse_q pass 1 lse, NLL, f = 1 / sum and the dX factor per row; the label
+//                column of P patched so that G = (dloss / N) diag(f) P;
+//                Xs = bf16(f X_b).  Rows whose logits leave the range R = 0
+//                serves are flagged instead
+//   repair GEMM  the forward GEMM again, only for the flagged 32-row groups,
+//                against each row's exact maximum (returns at once when
+//                nothing is flagged)
+//   lse_q pass 2 the flagged rows as in pass 1
+//   dX GEMM      dX_b = f (dloss / N) (P W)   (K = all of V; bf16 out)
+//   dW GEMM      dW  (+)= (dloss / N) P^T Xs  (fp32 running sum over chunks,
+//                bf16 -- or the fp32 sum -- on the last chunk)
+// then the loss over all rows.  P is never rewritten in full: the only pass
+// over it besides the two GEMMs that read it is one bf16 store per row.
+// Labels were checked by the caller.
 flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, const Ptrs& q,
                                     cudaStream_t st) {
   const int64_t BT = pl.BT, V = pl.V, H = pl.H;
@@ -770,7 +792,11 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
   float* rowloss = reinterpret_cast<float*>(q.ws + pl.off_rowloss);
   float* lse = reinterpret_cast<float*>(q.ws + pl.off_lse);
   __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(q.ws + pl.off_p);
-  CUtensorMap mx_k, mw_k, mw_mn, mx_mn, mdw_out;
+  __nv_bfloat16* Xs = reinterpret_cast<__nv_bfloat16*>(q.ws + pl.off_xs);
+  float* ref = reinterpret_cast<float*>(q.ws + pl.off_ref);
+  float* row_scale = reinterpret_cast<float*>(q.ws + pl.off_rowscale);
+  int* flags = reinterpret_cast<int*>(q.ws + pl.off_flags);
+  CUtensorMap mx_k, mw_k, mw_mn, mdw_out;
   // dW's map: bf16 pieces of 64 columns, or fp32 pieces of 32 when dW is fp32
   const bool ok_dw = pl.dw_f32 ? make_map(&mdw_out, q.dW, H, V, pl.lddw * 4, 32, 32,
                                           CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
@@ -778,18 +804,18 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
   if (!(ok_dw &&
         make_map(&mx_k, q.X, H, BT, pl.ldx * 2, 64, kBM) &&
         make_map(&mw_k, q.W, H, V, pl.ldw * 2, 64, b_box_rows()) &&
-        make_map(&mw_mn, q.W, H, V, pl.ldw * 2, 64, 64) &&
-        make_map(&mx_mn, q.X, H, BT, pl.ldx * 2, 64, 64)))
+        make_map(&mw_mn, q.W, H, V, pl.ldw * 2, 64, 64)))
     return FLCE_ERR_CUDA;
   const int sms = device_sms();
   const float cap = softcap_on(p->softcap) ? p->softcap : 0.f;
   for (int64_t b = 0; b < pl.n_row_chunks; ++b) {
     const int64_t row0 = b * pl.Cb;
     const int64_t rows = (BT - row0) < pl.Cb ? (BT - row0) : pl.Cb;
-    CUtensorMap mp_k, mp_mn, mp_out, mdx_out;
+    CUtensorMap mp_k, mp_mn, mp_out, mdx_out, mxs_mn;
     if (!(make_map(&mp_k, P, pl.ldp, rows, pl.ldp * 2, 64, kBM) &&
           make_map(&mp_mn, P, pl.ldp, rows, pl.ldp * 2, 64, 64) &&
           make_map(&mp_out, P, pl.ldp, rows, pl.ldp * 2, 64, 32) &&
+          make_map(&mxs_mn, Xs, H, rows, H * 2, 64, 64) &&
           make_map(&mdx_out, static_cast<__nv_bfloat16*>(q.dX) + row0 * pl.lddx, H, rows,
                    pl.lddx * 2, 64, 32)))
       return FLCE_ERR_CUDA;
@@ -803,17 +829,31 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     GemmArgs gf{rows, V, H, true};
     gf.wide_epi = pl.part_shift == 7;
     gf.a_mn_off = int(row0);
-    if (ep.softcap > 0.f)
-      FLCE_TRY((launch_gemm<false, false, EPI_LSE_P_CAP>(mx_k, mw_k, mp_out, gf, ep, sms, st)));
-    else
-      FLCE_TRY((launch_gemm<false, false, EPI_LSE_P>(mx_k, mw_k, mp_out, gf, ep, sms, st)));
-    prof_before(st);
-    lse_grad_kernel<<<unsigned(rows), kLseGradThreads, 0, st>>>(
-        partial, int(pl.part_tiles), pl.part_shift, BT, row0, target, q.labels, p->ignore_index,
-        pl.ldp, P, pl.ldp, lse, rowloss, hdr, q.dloss_host, cap);
-    prof_after(st, K_LSE_GRAD);
-    FLCE_TRY(cudaGetLastError());
-    // dX rows of this chunk: K runs over the whole vocabulary
+    const unsigned groups = unsigned(cdiv(rows, kLseQRows));
+    for (int pass = 1; pass <= 2; ++pass) {
+      TcEpi ef = ep;
+      if (pass == 2) {  // recompute only the flagged row groups
+        ef.ref = ref;
+        ef.row_group_flags = flags;
+        ef.n_groups = int(groups);
+      }
+      const int32_t kind = pass == 1 ? K_LSEQ_GEMM : K_LSEQ_REPAIR;
+      if (ef.softcap > 0.f)
+        FLCE_TRY((launch_gemm<false, false, EPI_LSE_Q_CAP>(mx_k, mw_k, mp_out, gf, ef, sms, st,
+                                                           kind)));
+      else
+        FLCE_TRY((launch_gemm<false, false, EPI_LSE_Q>(mx_k, mw_k, mp_out, gf, ef, sms, st,
+                                                       kind)));
+      prof_before(st);
+      lse_q_kernel<<<groups, kLseQThreads, 0, st>>>(
+          pass, partial, int(pl.part_tiles), BT, row0, rows, target, q.labels, p->ignore_index, P,
+          pl.ldp, static_cast<const __nv_bfloat16*>(q.X), pl.ldx, H, Xs, ref, flags, lse,
+          rowloss, row_scale, hdr, q.dloss_host, cap);
+      prof_after(st, K_LSEQ);
+      FLCE_TRY(cudaGetLastError());
+    }
+    // dX rows of this chunk: K runs over the whole vocabulary; each row
+    // scaled by its f dloss / N
     TcEpi ex = ep;
     ex.dx = static_cast<__nv_bfloat16*>(q.dX) + row0 * pl.lddx;
     ex.dx_first = 1;
@@ -821,6 +861,7 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     ex.dx_acc = reinterpret_cast<float*>(q.ws + pl.off_dxslab);
     ex.slab_stride = pl.Cb * H;
     ex.out_cols = int(H);
+    ex.row_scale = row_scale;
     GemmArgs gx{rows, H, round_up(V, 64), false};
     gx.k_splits = pl.dx_splits;
     FLCE_TRY((launch_gemm<false, true, EPI_DX>(mp_k, mw_mn, mdx_out, gx, ex, sms, st)));
@@ -830,12 +871,12 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
       if (blocks > 8 * sms) blocks = 8 * sms;
       prof_before(st);
       slab_reduce_kernel<<<blocks, 256, 0, st>>>(ex.dx_acc, pl.dx_splits, ex.slab_stride, n, H,
-                                                 ex.dx, pl.lddx, hdr);
+                                                 ex.dx, pl.lddx, row_scale, hdr);
       prof_after(st, K_DX_REDUCE);
       FLCE_TRY(cudaGetLastError());
     }
-    // dW += G_b^T X_b: an fp32 running sum over the row chunks, in the
-    // workspace, or in dW itself when dW is fp32
+    // dW += (dloss / N) P^T Xs: an fp32 running sum over the row chunks, in
+    // the workspace, or in dW itself when dW is fp32
     TcEpi ew = ep;
     ew.dx_acc = pl.dw_f32 ? static_cast<float*>(q.dW)
                           : reinterpret_cast<float*>(q.ws + pl.off_dwacc);
@@ -846,6 +887,9 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     ew.dx_first = b == 0;
     ew.dx_last = b == pl.n_row_chunks - 1;
     ew.out_cols = int(H);
+    ew.scale_by_nvalid = 1;
+    ew.n_valid = reinterpret_cast<const long long*>(q.ws + offsetof(WsHeader, n_valid));
+    ew.dloss_host = q.dloss_host;
     // The sum goes out by TMA stores: fp32 rows of the running sum, then dW
     // on the last chunk (bf16, or the fp32 sum itself).
     ew.tma_rmw = 1;
@@ -854,9 +898,8 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
                                  CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
       return FLCE_ERR_CUDA;
     GemmArgs gw{V, H, rows, false};
-    gw.b_k_off = int(row0);
-    FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mx_mn, ew.dx_last ? mdw_out : macc, gw, ew,
-                                              sms, st, K_DWACC_GEMM)));
+    FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, ew.dx_last ? mdw_out : macc, gw,
+                                              ew, sms, st, K_DWACC_GEMM)));
   }
   prof_before(st);
   finalize_kernel<<<1, 1024, 0, st>>>(rowloss, BT, hdr, q.loss);

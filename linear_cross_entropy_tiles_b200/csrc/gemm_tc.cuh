@@ -20,9 +20,10 @@
 //     EPI_DX   -- dX tile: fp32 accumulate across vocabulary chunks, bf16 on
 //                 the last chunk;
 //     EPI_DW   -- dW tile: bf16 store;
-//     EPI_LSE_P -- EPI_LSE for the fused-in-forward schedule: also stores
-//                 q = exp(y - m) * dy/dz (bf16) for every column, with the
-//                 (m, sum) partials that later turn q into G.
+//     EPI_LSE_Q -- EPI_LSE for the fused-in-forward schedule: also stores
+//                 q = exp(y - R) * dy/dz (bf16) for every column against one
+//                 reference R per row, with the (max, sum) partials; G is
+//                 then diag(f) q up to one scalar and the label column.
 // (_CAP variants apply the Gemma2 softcap.)
 //
 // Operands: A is M x K, B is N x K (D = A B^T).  Either may be K-major (rows
@@ -56,8 +57,8 @@ constexpr uint64_t kDrainLimitNs = 1000000000ull;
 // accumulates dW over row chunks in the fused-in-forward schedule.
 // The *_CAP modes are the same epilogues with the logit softcap compiled in.
 enum : int {
-  EPI_LSE = 0, EPI_GRAD = 1, EPI_DX = 2, EPI_DW = 3, EPI_LSE_P = 4,
-  EPI_LSE_CAP = 5, EPI_GRAD_CAP = 6, EPI_LSE_P_CAP = 7
+  EPI_LSE = 0, EPI_GRAD = 1, EPI_DX = 2, EPI_DW = 3, EPI_LSE_Q = 4,
+  EPI_LSE_CAP = 5, EPI_GRAD_CAP = 6, EPI_LSE_Q_CAP = 7
 };
 
 struct TcShape {
@@ -102,11 +103,23 @@ struct TcEpi {
   // (to dx_acc, which then is the output) instead of converting it.
   int out_f32;
   float* dw32;
-  // EPI_LSE_P (fused-in-forward schedule): rows of this launch start at row0;
-  // P is the chunk buffer [rows][ldp] of exp(y - reference), bf16
+  // EPI_LSE_Q (fused-in-forward schedule): rows of this launch start at row0;
+  // P is the chunk buffer [rows][ldp] of q = exp(y - R) dy/dz, bf16; ref, if
+  // set, holds each chunk row's exponent reference R (log2 units), else R = 0
   int64_t row0;
   __nv_bfloat16* P;
   int64_t ldp;
+  const float* ref;
+  // Any mode: if set, a work unit runs only when one of the 32-row groups of
+  // chunk rows its tile covers has a nonzero flag here (all roles skip the
+  // others alike); for recomputing the few rows whose logits left the
+  // shared reference's range.
+  const int* row_group_flags;
+  int n_groups;  // entries of row_group_flags
+  // EPI_DX: the result is multiplied by row_scale[row] (chunk rows) when set,
+  // and by dloss / N_valid (from n_valid, dloss_host) when scale_by_nvalid.
+  const float* row_scale;
+  int scale_by_nvalid;
   // bf16 output tiles stored by TMA: row added to the tile row (the
   // vocabulary offset of a dW chunk) and the output tensor's column count.
   int out_row_off;
@@ -219,6 +232,29 @@ __device__ __forceinline__ void tile_coords(const TcShape& sh, int t, int& mt, i
     nt = t % sh.n_tiles;
     mt = t / sh.n_tiles;
   }
+}
+
+// Whether any of the launch's row groups is flagged (every thread of the CTA
+// calls it once, in the prologue; true when no flags are given).
+__device__ __forceinline__ bool any_group_flagged(const TcEpi& ep) {
+  if (!ep.row_group_flags) return __syncthreads_or(1) != 0;
+  int any = 0;
+  for (int g = threadIdx.x; g < ep.n_groups; g += blockDim.x) any |= ep.row_group_flags[g];
+  return __syncthreads_or(any) != 0;
+}
+
+// Whether the work unit whose output rows are [m_lo, m_lo + rows) of the
+// launch runs: always, unless ep.row_group_flags asks for only the 32-row
+// groups flagged there (none at all: `any` is false and nothing runs).
+// Every role evaluates it for every unit alike.
+__device__ __forceinline__ bool tile_wanted(const TcEpi& ep, const TcShape& sh, int m_lo,
+                                            int rows, bool any = true) {
+  if (!ep.row_group_flags) return true;
+  if (!any) return false;
+  const int g1 = min(m_lo + rows, sh.M);
+  for (int g = m_lo; g < g1; g += 32)
+    if (ep.row_group_flags[g >> 5]) return true;
+  return false;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -424,6 +460,14 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
   float* slab = ep.dx_acc + int64_t(split) * ep.slab_stride + row * ep.H;
   // Otherwise a running sum in fp32 (streamed: read and written once per launch).
   float* accrow = ep.dx_acc + row * ep.ld_acc;
+  // The tile's factor (1 unless the launch asks for a row or global scale);
+  // K-split slabs stay unscaled, their reduction applies it.
+  float fac = 1.f;
+  if (ep.row_scale) fac = row_ok ? ep.row_scale[row] : 0.f;
+  if (ep.scale_by_nvalid) {
+    const long long nv = *ep.n_valid;
+    fac *= nv > 0 ? ep.dloss_host / float(nv) : 0.f;
+  }
 #pragma unroll 1
   for (int gq = c_lo * 32 / kLoadCols; gq < c_hi * 32 / kLoadCols; ++gq) {
     uint32_t vg[kLoadCols];
@@ -437,14 +481,15 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
         if (ep.out_f32) {
           float a[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(v[k]);
+          for (int k = 0; k < 32; ++k) a[k] = __uint_as_float(v[k]) * fac;
           put_f32(tma, c, a);
           continue;
         }
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          packed[k] = pack_bf16x2(__uint_as_float(v[2 * k]), __uint_as_float(v[2 * k + 1]));
+          packed[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * fac,
+                                  __uint_as_float(v[2 * k + 1]) * fac);
         put_bf16(tma, nullptr, c, packed);
         continue;
       }
@@ -459,10 +504,10 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
           float4 pv = make_float4(0.f, 0.f, 0.f, 0.f);
           if (row_ok && !ep.dx_first && c0 + 4 * g < ep.H)
             pv = __ldcs(reinterpret_cast<const float4*>(accrow + c0 + 4 * g));
-          a[4 * g] = __uint_as_float(v[4 * g]) + pv.x;
-          a[4 * g + 1] = __uint_as_float(v[4 * g + 1]) + pv.y;
-          a[4 * g + 2] = __uint_as_float(v[4 * g + 2]) + pv.z;
-          a[4 * g + 3] = __uint_as_float(v[4 * g + 3]) + pv.w;
+          a[4 * g] = fmaf(__uint_as_float(v[4 * g]), fac, pv.x);
+          a[4 * g + 1] = fmaf(__uint_as_float(v[4 * g + 1]), fac, pv.y);
+          a[4 * g + 2] = fmaf(__uint_as_float(v[4 * g + 2]), fac, pv.z);
+          a[4 * g + 3] = fmaf(__uint_as_float(v[4 * g + 3]), fac, pv.w);
         }
         if (!ep.dx_last || ep.out_f32) {
           put_f32(tma, c, a);
@@ -498,10 +543,10 @@ __device__ __forceinline__ void epi_dx(const TcEpi& ep, const TcShape& sh, int m
       for (int g = 0; g < 8; ++g) {
         const int64_t col = col0 + 4 * g;
         if (col >= ep.H) break;
-        const float4 a = make_float4(__uint_as_float(v[4 * g]) + prev[g].x,
-                                     __uint_as_float(v[4 * g + 1]) + prev[g].y,
-                                     __uint_as_float(v[4 * g + 2]) + prev[g].z,
-                                     __uint_as_float(v[4 * g + 3]) + prev[g].w);
+        const float4 a = make_float4(fmaf(__uint_as_float(v[4 * g]), fac, prev[g].x),
+                                     fmaf(__uint_as_float(v[4 * g + 1]), fac, prev[g].y),
+                                     fmaf(__uint_as_float(v[4 * g + 2]), fac, prev[g].z),
+                                     fmaf(__uint_as_float(v[4 * g + 3]), fac, prev[g].w));
         if (!ep.dx_last || ep.out_f32) {
           __stcs(reinterpret_cast<float4*>(accrow + col), a);
         } else {
@@ -567,76 +612,17 @@ __device__ __forceinline__ void epi_dw(const TcEpi& ep, const TcShape& sh, int m
   }
 }
 
-// Two passes over one warp's columns [c_lo, c_hi) of the tile: the exact
-// max of y, then q = exp(y - max).  MASK: some columns lie past the
-// vocabulary (ncols); full ranges are compiled without any per-column test.
-template <int BN, bool CAP, bool MASK>
-__device__ __forceinline__ void epi_lse_p_twopass(const TcEpi& ep, int64_t lrow, bool row_ok,
-                                              int lab_col, int ncols, uint32_t taddr,
-                                              TmaSink* tma, int c_lo, int c_hi, float* m_out,
-                                              float* s_out, float* tgt_out) {
-  const float sc = ep.softcap;
-  const float inv_sc = CAP ? 1.f / ep.softcap : 0.f;
-  float zmax = -INFINITY;
-#pragma unroll 1
-  for (int c = c_lo; c < c_hi; ++c) {
-    uint32_t v[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      if (!MASK || c * 32 + k < ncols) zmax = fmaxf(zmax, __uint_as_float(v[k]));
-  }
-  float dd;
-  const float m = capped<CAP>(zmax, sc, inv_sc, &dd) * kLog2e;
-  // Four running sums (fixed order, short dependency chains).
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, tgt = 0.f;
-  __nv_bfloat16* prow = ep.P + lrow * ep.ldp;
-#pragma unroll 1
-  for (int c = c_lo; c < c_hi; ++c) {
-    uint32_t v[32];
-    tmem_ld_32x32b_x32(taddr + c * 32, v);
-    tmem_ld_wait();
-    bool mine;
-    if (label_in_chunk(lab_col, c * 32, &mine) && mine) {
-      float d;
-      tgt = capped<CAP>(pick32(v, lab_col - c * 32), sc, inv_sc, &d);
-    }
-    uint32_t packed[16];
-#pragma unroll
-    for (int k = 0; k < 32; k += 2) {
-      float pv[2], qv[2];
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        float d;
-        const float y = capped<CAP>(__uint_as_float(v[k + e]), sc, inv_sc, &d);
-        pv[e] = ex2a(fmaf(y, kLog2e, -m));
-        if (MASK && c * 32 + k + e >= ncols) pv[e] = 0.f;
-        qv[e] = CAP ? pv[e] * d : pv[e];
-      }
-      if ((k & 2) == 0) {
-        a0 += pv[0];
-        a1 += pv[1];
-      } else {
-        a2 += pv[0];
-        a3 += pv[1];
-      }
-      packed[k / 2] = pack_bf16x2(qv[0], qv[1]);
-    }
-    put_bf16(tma, row_ok ? prow : nullptr, c, packed);
-  }
-  *m_out = m;
-  *s_out = (a0 + a1) + (a2 + a3);
-  *tgt_out = tgt;
-}
-
-// One 32-column chunk of the one-pass q epilogue: q for its columns (bf16,
-// through the sink), the running sums and, if the label column is here, its
-// y.  m is the exponent reference in log2 units.
+// One 32-column chunk of the fused-in-forward epilogue: for each column
+// q = exp2(y log2(e) - R) * dy/dz as bf16 through the sink (0 for a row whose
+// label is ignored), the running maximum of y and sum of exp2(y log2(e) - R),
+// and y at the label column if it lies here.  MASK: some
+// columns lie past the vocabulary (ncols); full ranges compile without the
+// per-column test.
 template <bool CAP, bool MASK>
-__device__ __forceinline__ void lse_p_chunk(const uint32_t (&cur)[32], int c, float m, float sc,
-                                            float inv_sc, int lab_col, int ncols, TmaSink* tma,
-                                            __nv_bfloat16* prow, float (&a)[4], float& tgt) {
+__device__ __forceinline__ void lse_q_chunk(const uint32_t (&cur)[32], int c, float R, float sc,
+                                            float inv_sc, int lab_col, bool keep, int ncols,
+                                            TmaSink* tma, __nv_bfloat16* prow, float (&a)[4],
+                                            float& mx, float& tgt) {
   bool mine;
   if (label_in_chunk(lab_col, c * 32, &mine) && mine) {
     float d;
@@ -650,9 +636,10 @@ __device__ __forceinline__ void lse_p_chunk(const uint32_t (&cur)[32], int c, fl
     for (int e = 0; e < 2; ++e) {
       float d;
       const float y = capped<CAP>(__uint_as_float(cur[k + e]), sc, inv_sc, &d);
-      pv[e] = ex2a(fmaf(y, kLog2e, -m));
-      if (MASK && c * 32 + k + e >= ncols) pv[e] = 0.f;
-      qv[e] = CAP ? pv[e] * d : pv[e];
+      const bool in = !MASK || c * 32 + k + e < ncols;
+      mx = in ? fmaxf(mx, y) : mx;  // in y; the caller scales it by log2(e)
+      pv[e] = in ? ex2a(fmaf(y, kLog2e, -R)) : 0.f;
+      qv[e] = keep ? (CAP ? pv[e] * d : pv[e]) : 0.f;
     }
     a[(k & 2) + 0] += pv[0];
     a[(k & 2) + 1] += pv[1];
@@ -661,102 +648,87 @@ __device__ __forceinline__ void lse_p_chunk(const uint32_t (&cur)[32], int c, fl
   put_bf16(tma, prow, c, packed);
 }
 
-// One pass over the same columns: the reference is the largest y of the
-// first 32-column chunk instead of the exact max.  Any reference works for
-// the (reference, sum) partial and for q, which bf16 holds over fp32's
-// exponent range; columns far below it flush to zero exactly as below the
-// true max.  Returns false when some column exceeded the reference by so
-// much that the sum reached 2^126 (every q below it is a finite bf16; the
-// two-pass version then redoes the range), or is NaN.  NCH = c_hi - c_lo
-// chunks (even), handled two per iteration: the TMEM load of the next chunk
-// is in flight while the current one is processed.
-template <int BN, bool CAP, bool MASK, int NCH>
-__device__ __forceinline__ bool epi_lse_p_onepass(const TcEpi& ep, int64_t lrow, bool row_ok,
-                                                  int lab_col, int ncols, uint32_t taddr,
-                                                  TmaSink* tma, int c_lo, float* m_out,
-                                                  float* s_out, float* tgt_out) {
+// One pass over a warp's columns [c_lo, c_lo + NCH) of the tile, two chunks
+// per iteration so the TMEM load of the next chunk is in flight while the
+// current one is processed.
+template <bool CAP, bool MASK, int NCH>
+__device__ __forceinline__ void epi_lse_q_range(const TcEpi& ep, float R, bool keep, int lab_col,
+                                                int ncols, uint32_t taddr, TmaSink* tma,
+                                                __nv_bfloat16* prow, int c_lo, float* m_out,
+                                                float* s_out, float* tgt_out) {
   static_assert(NCH % 2 == 0, "chunks are handled in pairs");
   const float sc = ep.softcap;
   const float inv_sc = CAP ? 1.f / ep.softcap : 0.f;
-  // Four running sums (fixed order, short dependency chains).
-  float a[4] = {0.f, 0.f, 0.f, 0.f};
-  float tgt = 0.f;
-  __nv_bfloat16* prow = row_ok ? ep.P + lrow * ep.ldp : nullptr;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};  // four running sums: fixed order, short chains
+  float mx = -INFINITY, tgt = 0.f;
   uint32_t v0[32], v1[32];
   tmem_ld_32x32b_x32(taddr + c_lo * 32, v0);
   tmem_ld_wait_regs(v0);
-  float m;
-  {
-    float zmax = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      if (!MASK || c_lo * 32 + k < ncols) zmax = fmaxf(zmax, __uint_as_float(v0[k]));
-    float dd;
-    m = capped<CAP>(zmax, sc, inv_sc, &dd) * kLog2e;
-  }
 #pragma unroll 1
   for (int i = 0; i < NCH; i += 2) {
     const int c = c_lo + i;
     tmem_ld_32x32b_x32(taddr + (c + 1) * 32, v1);
-    lse_p_chunk<CAP, MASK>(v0, c, m, sc, inv_sc, lab_col, ncols, tma, prow, a, tgt);
+    lse_q_chunk<CAP, MASK>(v0, c, R, sc, inv_sc, lab_col, keep, ncols, tma, prow, a, mx, tgt);
     __syncwarp();
     tmem_ld_wait_regs(v1);
     const bool more = i + 2 < NCH;
     if (more) tmem_ld_32x32b_x32(taddr + (c + 2) * 32, v0);
-    lse_p_chunk<CAP, MASK>(v1, c + 1, m, sc, inv_sc, lab_col, ncols, tma, prow, a, tgt);
+    lse_q_chunk<CAP, MASK>(v1, c + 1, R, sc, inv_sc, lab_col, keep, ncols, tma, prow, a, mx,
+                           tgt);
     if (more) {
       __syncwarp();
       tmem_ld_wait_regs(v0);
     }
   }
-  *m_out = m;
+  *m_out = mx * kLog2e;  // largest y, in log2 units
   *s_out = (a[0] + a[1]) + (a[2] + a[3]);
   *tgt_out = tgt;
-  // A column past the vocabulary has the reference -inf when the whole range
-  // is padding; its sum is 0 and nothing is stored from it.
-  return *s_out < 0x1p126f || (MASK && ncols <= c_lo * 32);
 }
 
-// Fused-in-forward variant of the LSE epilogue.  Pass 1 finds the tile's row
-// max from the raw logits (c*tanh(z/c) is increasing in z, so the max of y is
-// the cap of the max of z); pass 2 writes q = exp(y - max) * dy/dz for every
-// column as bf16 into the chunk buffer (dy/dz = 1 - tanh^2(z/c) under a
-// softcap, else 1) and sums the unrounded exp(y - max).  The (max, sum) pair
-// per (tile, row) both builds the lse and later rescales q into G.
+// Fused-in-forward epilogue.  Every row of the chunk shares one exponent
+// reference R (log2 units) across all its vocabulary tiles -- 0, or for a
+// row being recomputed because its logits left [-64, 64] (see lse_q_kernel)
+// the row's exact maximum from ep.ref -- so that G = (dloss / N) diag(f) Q
+// with one factor f_i = exp2(R_i - lse_i log2 e) per row, which the dX
+// epilogue and the prescaled X of the dW GEMM apply: the chunk buffer is
+// never rewritten.  Stores q = exp2(y log2 e - R) * dy/dz (bf16) for every
+// column, zeros for ignored rows, and per (slice, row) the partial (largest
+// y log2 e, sum of exp2(y log2 e - R)) plus the label's y.
+// The label of the row this thread drains in the tile starting at chunk row
+// m0, loaded before the accumulator is ready (its latency then hides behind
+// the wait); ignore_index past the chunk.
+__device__ __forceinline__ int64_t epi_row_label(const TcEpi& ep, const TcShape& sh, int m0,
+                                                 int r) {
+  const int64_t lrow = int64_t(m0) + r;
+  return lrow < sh.M ? __ldg(ep.labels + ep.row0 + lrow) : ep.ignore_index;
+}
+
 template <int BN, bool CAP, int NCH = BN / 32>
-__device__ __forceinline__ void epi_lse_p(const TcEpi& ep, const TcShape& sh, int m0, int n0,
+__device__ __forceinline__ void epi_lse_q(const TcEpi& ep, const TcShape& sh, int m0, int n0,
                                           int part, int r, uint32_t taddr,
                                           TmaSink* tma = nullptr, int c_lo = 0,
-                                          int c_hi = BN / 32) {
+                                          int c_hi = BN / 32, int64_t lab_pre = INT64_MIN) {
   const int64_t lrow = int64_t(m0) + r;  // row within the chunk
+  // A recomputation touches only the flagged 32-row groups: exactly this
+  // warp's rows (warp-uniform), so the rows of other groups keep what the
+  // first pass and its finishing kernel wrote.
+  if (ep.row_group_flags && ep.row_group_flags[lrow >> 5] == 0) return;
   const int64_t row = ep.row0 + lrow;    // row of X
   const bool row_ok = lrow < sh.M;
-  const int64_t lab = row_ok ? __ldg(ep.labels + row) : ep.ignore_index;
-  const int lab_col = (lab != ep.ignore_index && lab >= n0 && lab < int64_t(n0) + BN)
-                          ? int(lab - n0) : -1;
+  const int64_t lab = lab_pre != INT64_MIN ? lab_pre : epi_row_label(ep, sh, m0, r);
+  const bool keep = lab != ep.ignore_index;
+  const int lab_col = (keep && lab >= n0 && lab < int64_t(n0) + BN) ? int(lab - n0) : -1;
   const int ncols = sh.N - n0;  // columns of this tile inside the vocabulary
-  TcEpi e2 = ep;
-  e2.P = ep.P + n0;
+  const float R = (ep.ref && row_ok) ? ep.ref[lrow] : 0.f;
+  __nv_bfloat16* prow = row_ok ? ep.P + lrow * ep.ldp + n0 : nullptr;
   float m, s, tgt;
-  const bool full = ncols >= c_hi * 32;
-  bool ok = full ? epi_lse_p_onepass<BN, CAP, false, NCH>(e2, lrow, row_ok, lab_col, ncols,
-                                                          taddr, tma, c_lo, &m, &s, &tgt)
-                 : epi_lse_p_onepass<BN, CAP, true, NCH>(e2, lrow, row_ok, lab_col, ncols, taddr,
-                                                         tma, c_lo, &m, &s, &tgt);
-  if (!__all_sync(0xffffffffu, ok)) {
-    // Rare: redo the warp's range with the exact max.  Its earlier stores of
-    // the same q pieces must land first.
-    if (tma) {
-      if (tma->lane == 0) bulk_wait_group<0>();
-      __syncwarp();
-    }
-    if (full)
-      epi_lse_p_twopass<BN, CAP, false>(e2, lrow, row_ok, lab_col, ncols, taddr, tma, c_lo,
-                                        c_hi, &m, &s, &tgt);
-    else
-      epi_lse_p_twopass<BN, CAP, true>(e2, lrow, row_ok, lab_col, ncols, taddr, tma, c_lo, c_hi,
-                                       &m, &s, &tgt);
-  }
+  if (ncols >= c_hi * 32)
+    epi_lse_q_range<CAP, false, NCH>(ep, R, keep, lab_col, ncols, taddr, tma, prow, c_lo, &m,
+                                     &s, &tgt);
+  else
+    epi_lse_q_range<CAP, true, NCH>(ep, R, keep, lab_col, ncols, taddr, tma, prow, c_lo, &m, &s,
+                                    &tgt);
+  // Columns wholly past the vocabulary form no partial.
   if (row_ok && ncols > c_lo * 32) {
     ep.partial[size_t(part) * size_t(ep.BT) + size_t(row)] = make_float2(m, s);
     if (lab_col >= c_lo * 32 && lab_col < c_hi * 32) ep.target[row] = tgt;
@@ -824,7 +796,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const bool skip = *abort_flag != 0;  // an earlier kernel of this call failed
+  const bool any = any_group_flagged(ep);  // a recomputation with nothing flagged: no units
+  const bool skip = *abort_flag != 0 || !any;  // (or an earlier kernel of this call failed)
   const uint64_t limit = ep.wait_limit_ns;
 
   if (!skip && warp == 0 && lane == 0) {
@@ -840,6 +813,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int t = blockIdx.x; ok && t < sh.num_tiles; t += gridDim.x) {
       int mt, nt;
       tile_coords(sh, t, mt, nt);
+      if (!tile_wanted(ep, sh, mt * kBM, kBM)) continue;
       const int m0 = mt * kBM + sh.a_mn_off;
       const int n0 = nt * BN + sh.b_mn_off;
       for (int kb = 0; kb < sh.k_blocks; ++kb) {
@@ -884,6 +858,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t s = 0, ph = 0, acc = 0, aph = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < sh.num_tiles; t += gridDim.x) {
+      {
+        int mt, nt;
+        tile_coords(sh, t, mt, nt);
+        if (!tile_wanted(ep, sh, mt * kBM, kBM)) continue;
+      }
       if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, limit, abort_flag)) {
         record_timeout(ep, abort_flag);
         ok = false;
@@ -930,6 +909,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int t = blockIdx.x; t < sh.num_tiles; t += gridDim.x) {
       int mt, nt;
       tile_coords(sh, t, mt, nt);
+      if (!tile_wanted(ep, sh, mt * kBM, kBM)) continue;
       // Every lane polls; all must agree before the warp-wide tcgen05.ld.
       const bool got = mbar_wait_bounded(&tfull[acc], aph, limit, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
@@ -946,8 +926,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (MODE == EPI_GRAD_CAP) epi_grad<BN, true>(ep, sh, m0, n0, r, taddr);
       if (MODE == EPI_DX) epi_dx<BN>(ep, sh, m0, n0, r, taddr);
       if (MODE == EPI_DW) epi_dw<BN>(ep, sh, m0, n0, r, taddr);
-      if (MODE == EPI_LSE_P) epi_lse_p<BN, false>(ep, sh, m0, n0, nt, r, taddr);
-      if (MODE == EPI_LSE_P_CAP) epi_lse_p<BN, true>(ep, sh, m0, n0, nt, r, taddr);
+      if (MODE == EPI_LSE_Q) epi_lse_q<BN, false>(ep, sh, m0, n0, nt, r, taddr);
+      if (MODE == EPI_LSE_Q_CAP) epi_lse_q<BN, true>(ep, sh, m0, n0, nt, r, taddr);
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       acc ^= 1u;

@@ -116,7 +116,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc2_threads(EW), 1)
   cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const bool skip = *abort_flag != 0;
+  // A recomputation with no row group flagged has no work units; both CTAs
+  // of the pair read the same flags and agree.
+  const bool skip = *abort_flag != 0 || !any_group_flagged(ep);
   const uint64_t limit = ep.wait_limit_ns;
 
   if (!skip && warp == 0 && lane == 0) {
@@ -132,6 +134,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc2_threads(EW), 1)
       const int split = u / sh.num_tiles;
       int mt, nt;
       tile_coords(sh, u - split * sh.num_tiles, mt, nt);
+      if (!tile_wanted(ep, sh, mt * kPairBM, kPairBM)) continue;
       const int m0 = mt * kPairBM + 128 * int(rank) + sh.a_mn_off;
       const int n0 = nt * kPairBN + 128 * int(rank) + sh.b_mn_off;
       const int kb1 = min(k_stages, (split + 1) * kps);
@@ -184,6 +187,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc2_threads(EW), 1)
     bool ok = true;
     for (int u = pair; ok && u < n_units; u += n_pairs) {
       const int split = u / sh.num_tiles;
+      {
+        int mt, nt;
+        tile_coords(sh, u - split * sh.num_tiles, mt, nt);
+        if (!tile_wanted(ep, sh, mt * kPairBM, kPairBM)) continue;
+      }
       if (!mbar_wait_bounded(&tempty[acc], aph ^ 1u, limit, abort_flag)) {
         record_timeout(ep, abort_flag);
         ok = false;
@@ -247,6 +255,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc2_threads(EW), 1)
       const int split = u / sh.num_tiles;
       int mt, nt;
       tile_coords(sh, u - split * sh.num_tiles, mt, nt);
+      if (!tile_wanted(ep, sh, mt * kPairBM, kPairBM)) continue;
+      constexpr bool kQ = MODE == EPI_LSE_Q || MODE == EPI_LSE_Q_CAP;
+      const int64_t lab_pre =
+          kQ ? epi_row_label(ep, sh, mt * kPairBM + 128 * int(rank), q * 32 + lane) : 0;
       const bool got = mbar_wait_bounded(&tfull[acc], aph, limit, abort_flag);
       if (!__all_sync(0xffffffffu, got)) {
         if (lane == 0) record_timeout(ep, abort_flag);
@@ -270,10 +282,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc2_threads(EW), 1)
       if (MODE == EPI_DX)
         epi_dx<BN, EW == 8 ? 64 : 128>(ep, sh, m0, n0, r, taddr, split, &sink, c_lo, c_hi);
       if (MODE == EPI_DW) epi_dw<BN>(ep, sh, m0, n0, r, taddr, &sink, c_lo, c_hi);
-      if (MODE == EPI_LSE_P)
-        epi_lse_p<BN, false, kChunks>(ep, sh, m0, n0, part, r, taddr, &sink, c_lo, c_hi);
-      if (MODE == EPI_LSE_P_CAP)
-        epi_lse_p<BN, true, kChunks>(ep, sh, m0, n0, part, r, taddr, &sink, c_lo, c_hi);
+      if (MODE == EPI_LSE_Q)
+        epi_lse_q<BN, false, kChunks>(ep, sh, m0, n0, part, r, taddr, &sink, c_lo, c_hi,
+                                      lab_pre);
+      if (MODE == EPI_LSE_Q_CAP)
+        epi_lse_q<BN, true, kChunks>(ep, sh, m0, n0, part, r, taddr, &sink, c_lo, c_hi,
+                                     lab_pre);
       tc_fence_before();
       mbar_arrive_cluster(mapa_shared(&tempty[acc], 0));
       acc ^= 1u;

@@ -93,6 +93,10 @@ def test_fused_dp_one_rank_nccl_equals_fused(cuda_device):
         ref = flce.fused(X, W, lab)
         torch.cuda.synchronize()
         assert int(n.item()) == int((lab != -100).sum().item())
-        assert torch.equal(loss, ref[0]) and torch.equal(dX, ref[1]) and torch.equal(dW, ref[2])
+        assert dW.dtype == torch.float32           # summed over ranks in fp32
+        assert torch.equal(loss, ref[0]) and torch.equal(dX, ref[1])
+        assert torch.equal(dW.to(torch.bfloat16), ref[2])
+        l16, dX16, dW16, _ = dp.fused_dp(X, W, lab, dw_fp32=False)
+        assert dW16.dtype == torch.bfloat16 and torch.equal(dW16, ref[2])
     finally:
         dist.destroy_process_group()

@@ -72,7 +72,9 @@ def test_workspace_cap_keeps_results(cap_kind, cuda_device):
     """Under a cap the automatic schedule switches to the recompute plan (and
     narrows its vocabulary chunk for the tiny cap): results match the oracle,
     and the workspace the caller allocates is the capped size."""
-    BT, H, V = 1024, 128, 6000
+    # H > BT / 2: the fused-in-forward plan's fp32 dW sum (V x H) alone is
+    # larger than one bf16 BT x V tensor, so the logits-sized cap rejects it
+    BT, H, V = 1024, 1024, 6000
     X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.05, 0.1, seed=53, device=cuda_device)
     p = flce.make_problem(BT, H, V, X.dtype)
     cap = 2 * BT * V if cap_kind == "logits" else 1

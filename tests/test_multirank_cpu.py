@@ -126,3 +126,57 @@ def test_data_parallel_step_gloo_world2():
             assert torch.allclose(loss, ref_loss, rtol=1e-12, atol=1e-14)
             assert torch.allclose(dW, ref_dW, rtol=1e-12, atol=1e-14)
             assert torch.allclose(dX, ref_dX[rows], rtol=1e-12, atol=1e-14)
+
+
+def _dw_reduce_worker(rank, world, port, q, shares):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from linear_cross_entropy_tiles_b200 import dp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        out = {}
+        for dt in (torch.float32, torch.bfloat16):
+            share = shares[rank].to(dt)
+            _, _, dW, _ = dp.data_parallel_step(
+                lambda: torch.ones(1, dtype=torch.int64),
+                lambda n: (torch.zeros(1), torch.zeros(1), share.clone()))
+            out[str(dt)] = dW.float().numpy().copy()
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_dw_summed_over_ranks_in_fp32(world):
+    """Each rank's dW share in fp32 (what dp.fused_dp has the library write)
+    summed by the collective in fp32: every rank gets the same sum, within
+    fp32 rounding of the exact (fp64) sum of the shares.  The same shares
+    rounded to bf16 and summed in bf16 are off by bf16's 8-bit rounding,
+    hundreds of times more: why the fp32 reduction is the default."""
+    g = torch.Generator().manual_seed(11)
+    shares = [torch.randn(64, 48, generator=g, dtype=torch.float64) * 1e-3
+              for _ in range(world)]
+    exact = sum(shares)
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_dw_reduce_worker, args=(r, world, port, q, shares))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    ref = exact.numpy()
+    scale = float(abs(ref).max())
+    f32 = [got[r]["torch.float32"] for r in range(world)]
+    b16 = [got[r]["torch.bfloat16"] for r in range(world)]
+    assert all((f == f32[0]).all() for f in f32) and all((b == b16[0]).all() for b in b16)
+    err32 = float(abs(f32[0] - ref).max()) / scale
+    err16 = float(abs(b16[0] - ref).max()) / scale
+    assert err32 <= world * 2.0 ** -23
+    assert err16 >= 100 * err32 and err16 <= world * 2.0 ** -8

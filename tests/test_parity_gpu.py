@@ -171,10 +171,11 @@ def test_launch_count_and_stream(cuda_device):
         flce.fused(Xd, Wd, labd)
         n = flce.flce_last_launch_count()
         names = [k for k, _ in flce.flce_profile_stop()]
-    # labels, 2 row chunks x (LSE+p GEMM, lse_grad, dX GEMM [+ split reduce],
-    # dW GEMM), finalize
+    # labels, 2 row chunks x (forward GEMM, lse_q, recomputation GEMM (returns
+    # at once: nothing flagged), lse_q, dX GEMM [+ split reduce], dW GEMM),
+    # finalize
     assert len(names) == n
-    chunk = ["lse_p_gemm", "lse_grad", "dx_gemm"]
+    chunk = ["lse_q_gemm", "lse_q", "lse_q_repair_gemm", "lse_q", "dx_gemm"]
     tail = ["dw_acc_gemm"]
     body = names[1:-1]
     if "dx_reduce" in body:
@@ -300,3 +301,40 @@ def test_cuda_graph_capture_and_replay(sched, cuda_device):
             assert torch.equal(loss, ref[0]) and torch.equal(dX, ref[1])
             assert torch.equal(dW, ref[2])
             Xd.mul_(0.5)  # new inputs in the same buffers
+
+
+@pytest.mark.parametrize("cap", [0.0, 60.0])
+@pytest.mark.parametrize("H", [64, 1096])
+def test_rows_outside_the_shared_reference_range(cap, H, cuda_device):
+    """The fused-in-forward schedule stores q = exp(y - R) against one
+    reference R = 0 per row.  Rows whose logits all sit near +80 nats (one
+    near +200, where the sums overflow) or near -80 nats leave the range that
+    keeps q and the prescaled X in bf16; they are flagged, their 32-row
+    groups recomputed against each row's own maximum, and the other rows of
+    those groups and tiles finished again with the same values.  Ignored
+    rows are never flagged.  Everything matches the oracle."""
+    BT, V = 700, 3000
+    X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.05, 0.1, 91)
+    W[:, 0] = 1.0     # X[i, 0] now shifts every logit of row i
+    X[:, 0] = 0.0
+    high, low = [5, 300, 301, 650], [70, 71, 400, 699]
+    X[high, 0] = 80.0
+    X[low, 0] = -80.0
+    X[130, 0] = 200.0
+    lab[[5, 71]] = inputs.IGNORE_INDEX
+    o = run_oracle(X, W, lab, softcap=cap, dloss=0.5)
+    with schedule(SCHEDULES["fused_fwd"]):
+        loss, dX, dW = flce.fused(X.to(cuda_device), W.to(cuda_device), lab.to(cuda_device),
+                                  softcap=cap, dloss=0.5)
+    torch.cuda.synchronize()
+    assert torch.isfinite(dX).all() and torch.isfinite(dW).all()
+    tol = TOL["bf16"]
+    assert rel_scalar(loss.item(), o["loss"]) <= tol["loss"], (loss.item(), o["loss"])
+    assert rel_fro(to_np(dX), o["dX"]) <= tol["grad"]
+    assert rel_fro(to_np(dW), o["dW"]) <= tol["grad"]
+    # row by row: the recomputed rows and their group neighbours
+    for i in high + low + [130, 131, 301, 64]:
+        ref = o["dX"][i]
+        nrm = np.linalg.norm(ref)
+        got = to_np(dX[i:i + 1])[0]
+        assert (nrm == 0 and not got.any()) or np.linalg.norm(got - ref) <= 2e-2 * nrm, i
