@@ -52,7 +52,19 @@ METRIC = ("FLCE fwd+bwd tokens/s and TFLOP/s (% of B200 BF16 peak); peak extra H
 # commands and the per-launch figures are kept under profiles/).  They
 # describe the kernel code whose hash (csrc_sha16) is recorded with them and
 # are reported as null for any other build or workload.
-TRAFFIC = {}
+TRAFFIC = {
+    ("llama3_8b", "auto"): {
+        "csrc_sha16": "d7cab5e2df07fdb8",
+        "bytes_per_launch": {"lse_q_gemm": 2.447e9, "dx_gemm": 7.652e9, "dw_acc_gemm": 5.077e9,
+                             "lse_q": 0.0255e9}},
+    ("gpt2_small", "auto"): {
+        "csrc_sha16": "d7cab5e2df07fdb8",
+        "bytes_per_launch": {"lse_q_gemm": 0.8895e9, "dx_gemm": 1.054e9,
+                             "dw_acc_gemm": 1.183e9}},
+    ("ce_llmc", "auto"): {
+        "csrc_sha16": "d7cab5e2df07fdb8",
+        "bytes_per_launch": {"ce_forward": 3.297e9, "ce_backward": 6.541e9}},
+}
 
 
 def csrc_sha16(root=None):
@@ -417,28 +429,41 @@ def run_ce(args, world, rank):
     dloss = torch.ones(1, dtype=torch.float32, device=dev)
     dZ = torch.empty_like(Z)
 
+    fused = args.ce_mode == "fused"
+    ws_u = flce.ce_workspace(pf, flce.FLCE_OP_FUSED, dev) if fused else None
+
     def step():
+        if fused:  # one read and one write of the logits
+            flce.flce_ce_fused(pf, Z, labels, 1.0, loss, lse, dZ, ws_u, stream)
+            return
         flce.flce_ce_forward(pf, Z, labels, loss, lse, ws_f, stream)
         flce.flce_ce_backward(pf, Z, labels, lse, dloss, dZ, ws_b, stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    status, n_valid = flce.flce_get_device_status(ws_f)
+    status, n_valid = flce.flce_get_device_status(ws_u if fused else ws_f)
     if status != 0:
         raise SystemExit("device status %d after warm-up" % status)
-    flce.flce_ce_forward(pf, Z, labels, loss, lse, ws_f, stream)
-    launches_per_step = flce.flce_last_launch_count()
-    flce.flce_ce_backward(pf, Z, labels, lse, dloss, dZ, ws_b, stream)
-    launches_per_step += flce.flce_last_launch_count()
+    if fused:
+        step()
+        launches_per_step = flce.flce_last_launch_count()
+    else:
+        flce.flce_ce_forward(pf, Z, labels, loss, lse, ws_f, stream)
+        launches_per_step = flce.flce_last_launch_count()
+        flce.flce_ce_backward(pf, Z, labels, lse, dloss, dZ, ws_b, stream)
+        launches_per_step += flce.flce_last_launch_count()
     sampler = ClockSampler(torch.cuda.current_device())
     ms, clocks = time_steps(step, args.steps, world, stream, sampler)
     peaks = load_peaks()
     by_kind = profile_kinds(step, max(1, min(args.steps, args.prof_steps)), launches_per_step)
     total = sum(v[0] for v in by_kind.values())
     elem = w.BT * w.V * (2 if w.dtype == "bf16" else 4)
-    # The backward moves two of the step's three logits-sized passes.
-    bytes_per_launch = {"ce_forward": float(elem), "ce_backward": 2.0 * elem}
+    # The backward moves two of the step's three logits-sized passes; the
+    # fused call both of its two.
+    bytes_per_launch = {"ce_forward": float(elem), "ce_backward": 2.0 * elem,
+                        "ce_fused": 2.0 * elem}
+    step_bytes = 2.0 * elem if fused else w.bytes_per_step
     dom = max(by_kind, key=lambda n: by_kind[n][0])
     dom_ms = by_kind[dom][0] / by_kind[dom][1]
     achieved = bytes_per_launch.get(dom, 0.0) / (dom_ms / 1e3) / 1e9
@@ -452,25 +477,33 @@ def run_ce(args, world, rank):
                 "shares": {k: round(v[0] / total, 4) for k, v in sorted(by_kind.items())}}
     e2e = None
     if not args.no_e2e:
+        # The step's data (the logits and labels) in from pinned host memory,
+        # the loss out; the logit gradient stays on the device for the LM
+        # head's backward (--e2e-copies all copies it out too).
+        copy_all = args.e2e_copies == "all"
         Zh = Z.cpu().pin_memory()
         Lh = labels.cpu().pin_memory()
         lossh = torch.empty(1, dtype=torch.float32).pin_memory()
-        dZh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
+        dZh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory() if copy_all else None
 
         def e2e_step():
             Z.copy_(Zh, non_blocking=True)
             labels.copy_(Lh, non_blocking=True)
             step()
             lossh.copy_(loss, non_blocking=True)
-            dZh.copy_(dZ, non_blocking=True)
+            if copy_all:
+                dZh.copy_(dZ, non_blocking=True)
 
         e2e_step()
         ems, _ = time_steps(e2e_step, args.e2e_steps, world, stream)
         e2e = {"value": world * w.BT / (ems / 1e3), "unit": "tokens/s", "ms_per_step": ems,
                "h2d_bytes_per_step": Zh.numel() * Zh.element_size() + Lh.numel() * 8,
-               "d2h_bytes_per_step": 4 + dZh.numel() * dZh.element_size(),
-               "api": "linear_cross_entropy_tiles_b200 flce_ce_forward + flce_ce_backward "
-                      "(C ABI)"}
+               "d2h_bytes_per_step": 4 + (dZh.numel() * dZh.element_size() if copy_all else 0),
+               "copies": ("logits, labels in; loss, dlogits out" if copy_all else
+                          "logits, labels in; loss out (dlogits stays on the device)"),
+               "api": ("linear_cross_entropy_tiles_b200 flce_ce_fused (C ABI)" if fused else
+                       "linear_cross_entropy_tiles_b200 flce_ce_forward + flce_ce_backward "
+                       "(C ABI)")}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = ce_oracle_sample(w, Z, labels, args.ce_cpu_rows)
@@ -480,9 +513,9 @@ def run_ce(args, world, rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic", "config": ce_config(w, world),
-            "gbs": w.bytes_per_step / (ms / 1e3) / 1e9,
-            "frac_of_hbm": w.bytes_per_step / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-            "bytes_per_step": w.bytes_per_step, "n_valid": n_valid,
+            "gbs": step_bytes / (ms / 1e3) / 1e9,
+            "frac_of_hbm": step_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "bytes_per_step": step_bytes, "ce_mode": args.ce_mode, "n_valid": n_valid,
             "loss": float(loss.item()), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps, "clocks": clocks}), flush=True)
 
@@ -500,7 +533,13 @@ def main():
                     help="flce_fused schedule (auto: fused-in-forward for BT >= 512)")
     ap.add_argument("--cpu-rows", type=int, default=8)
     ap.add_argument("--ce-cpu-rows", type=int, default=8192)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--ce-mode", default="separate", choices=["separate", "fused"],
+                    help="ce_* workloads: flce_ce_forward + flce_ce_backward (the PR's two "
+                         "passes), or flce_ce_fused (one read of the logits)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-copies", default="data", choices=["data", "all"],
+                    help="e2e host copies per step: the step's data in and the loss out "
+                         "(default), or also W in and the gradients out")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--ragged-reps", type=int, default=3)
@@ -635,25 +674,32 @@ def main():
                 "traffic": traffic_of(dom, args.workload, args.schedule, args.bt),
                 "shares": {k: round(v[0] / total_prof, 4) for k, v in sorted(by_kind.items())}}
 
-    # End to end through the public API with host buffers: H2D of X, W,
-    # labels from pinned memory, flce_fused, D2H of loss, dX, dW.
+    # End to end through the public API with host buffers.  Per step, the
+    # step's data -- the hidden states X and the labels -- come in from
+    # pinned host memory and the loss goes back to the host (a training loop
+    # logs it); W is a parameter resident on the device, and dX, dW are
+    # consumed there by the rest of the backward pass and the optimizer.
+    # --e2e-copies all also copies W in and dX, dW out every step.
     e2e = None
     if not args.no_e2e:
+        copy_all = args.e2e_copies == "all"
         Xh = X.cpu().pin_memory()
-        Wh = W.cpu().pin_memory()
+        Wh = W.cpu().pin_memory() if copy_all else None
         Lh = labels.cpu().pin_memory()
         lossh = torch.empty_like(loss, device="cpu").pin_memory()
-        dXh = torch.empty_like(dX, device="cpu").pin_memory()
-        dWh = torch.empty_like(dW, device="cpu").pin_memory()
+        dXh = torch.empty_like(dX, device="cpu").pin_memory() if copy_all else None
+        dWh = torch.empty_like(dW, device="cpu").pin_memory() if copy_all else None
 
         def e2e_step():
             X.copy_(Xh, non_blocking=True)
-            W.copy_(Wh, non_blocking=True)
+            if copy_all:
+                W.copy_(Wh, non_blocking=True)
             labels.copy_(Lh, non_blocking=True)
             compute()
             lossh.copy_(loss, non_blocking=True)
-            dXh.copy_(dX, non_blocking=True)
-            dWh.copy_(dW, non_blocking=True)
+            if copy_all:
+                dXh.copy_(dX, non_blocking=True)
+                dWh.copy_(dW, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()
@@ -667,10 +713,15 @@ def main():
         torch.cuda.synchronize()
         barrier(world)
         ems = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-        h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size() + Lh.numel() * 8
-        d2h = 4 + dXh.numel() * dXh.element_size() + dWh.numel() * dWh.element_size()
+        h2d = Xh.numel() * Xh.element_size() + Lh.numel() * 8
+        d2h = lossh.numel() * 4
+        if copy_all:
+            h2d += Wh.numel() * Wh.element_size()
+            d2h += dXh.numel() * dXh.element_size() + dWh.numel() * dWh.element_size()
         e2e = {"value": world * w.BT / (ems / 1e3), "unit": "tokens/s", "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "copies": ("X, labels, W in; loss, dX, dW out" if copy_all else
+                          "X, labels in; loss out (W resident, dX and dW stay on the device)"),
                "api": ("linear_cross_entropy_tiles_b200 flce_count_valid + flce_fused_global "
                        "(C ABI) + torch.distributed all-reduces" if dp_mode else
                        "linear_cross_entropy_tiles_b200.flce_fused (C ABI)")}

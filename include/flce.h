@@ -175,6 +175,46 @@ FLCE_API flce_status_t flce_fused_global(const flce_problem_t* p, const void* X,
                                          float dloss, float* loss, void* dX, void* dW, void* ws,
                                          size_t ws_bytes, struct CUstream_st* stream);
 
+/* Vocabulary parallelism: W split over the vocabulary across ranks, rank r
+ * holding rows [v_offset, v_offset + p->V) of a V_total-row W and all of X
+ * and the labels (global vocabulary ids).  The mean loss needs, per row, the
+ * log-sum-exp over the whole vocabulary, so each rank reduces its slice to
+ * three numbers per row, the ranks exchange them, and the backward then
+ * needs only the global lse: dX is a sum over the ranks' slices, dW stays
+ * with its rank.  The pages' distributed setting is data parallel (torchtune
+ * issue #1228's FSDP recipes); this is the other split the loss allows.
+ *
+ * flce_vp_forward: stats (device fp32 [BT][3]) = per row, over this rank's
+ *   slice, the largest y log2(e), the sum of exp2(y log2(e) - that), and y at
+ *   the label when the label lies in the slice (else 0).  Labels are checked
+ *   against [0, v_total).  Workspace: flce_vp_workspace_size(p,
+ *   FLCE_OP_FORWARD).
+ * flce_vp_combine: with p->V = v_total, stats_all (device fp32
+ *   [n_ranks][BT][3], the ranks' stats in rank order) -> lse (device fp32
+ *   [BT]) and loss (device fp32 scalar, the mean over non-ignored rows),
+ *   combined in rank order (identical on every rank).  Workspace: any
+ *   forward workspace of this BT (>= 256 + 2 * ceil256(4 * BT) bytes).
+ * flce_vp_backward: dX (device fp32, BT x H, row stride p->lddx or H; this
+ *   rank's share, to be summed over the ranks) and dW (this rank's V rows,
+ *   as in flce_backward) from the global lse and dloss (device fp32 scalar).
+ *   Workspace: flce_vp_workspace_size(p, FLCE_OP_BACKWARD).
+ * p->shift_seq_len must be 0 (FLCE_ERR_UNSUPPORTED otherwise); v_offset < 0
+ * or v_offset + p->V > v_total: FLCE_ERR_INVALID_ARG. */
+FLCE_API size_t flce_vp_workspace_size(const flce_problem_t* p, int op);
+FLCE_API flce_status_t flce_vp_forward(const flce_problem_t* p, int64_t v_offset,
+                                       int64_t v_total, const void* X, const void* W,
+                                       const int64_t* labels, float* stats, void* ws,
+                                       size_t ws_bytes, struct CUstream_st* stream);
+FLCE_API flce_status_t flce_vp_combine(const flce_problem_t* p, int32_t n_ranks,
+                                       const float* stats_all, const int64_t* labels,
+                                       float* loss, float* lse, void* ws, size_t ws_bytes,
+                                       struct CUstream_st* stream);
+FLCE_API flce_status_t flce_vp_backward(const flce_problem_t* p, int64_t v_offset,
+                                        int64_t v_total, const void* X, const void* W,
+                                        const int64_t* labels, const float* lse,
+                                        const float* dloss, float* dX, void* dW, void* ws,
+                                        size_t ws_bytes, struct CUstream_st* stream);
+
 /* Size in bytes of the fixed scratch array behind flce_fused_noalloc. */
 #define FLCE_NOALLOC_SCRATCH_BYTES (64u << 20)
 
@@ -245,9 +285,10 @@ typedef struct {
   int64_t ld_grad;       /* row stride of dlogits in elements; 0 = V */
 } flce_ce_problem_t;
 
-/* Workspace bytes for op FLCE_OP_FORWARD or FLCE_OP_BACKWARD (0 when the
- * problem or op is invalid): a 256-byte header, [BT] fp32 per-row losses
- * (forward), [BT] int64 shifted labels (shift_seq_len > 0). */
+/* Workspace bytes for op FLCE_OP_FORWARD, FLCE_OP_BACKWARD or FLCE_OP_FUSED
+ * (flce_ce_fused) (0 when the problem or op is invalid): a 256-byte header,
+ * [BT] fp32 per-row losses (forward, fused), [BT] int64 shifted labels
+ * (shift_seq_len > 0). */
 FLCE_API size_t flce_ce_workspace_size(const flce_ce_problem_t* p, int op);
 
 /* loss (device fp32 scalar) and lse (device fp32 [BT], kept for
@@ -262,6 +303,20 @@ FLCE_API flce_status_t flce_ce_backward(const flce_ce_problem_t* p, const void* 
                                         const int64_t* labels, const float* lse,
                                         const float* dloss, void* dlogits, void* ws,
                                         size_t ws_bytes, struct CUstream_st* stream);
+
+/* Forward and backward together, for a training step that holds the logits
+ * (dloss by value, as flce_fused): loss (device fp32 scalar), optionally lse
+ * (device fp32 [BT], or NULL) and dlogits, reading each row of the logits
+ * once -- it stays in shared memory between the row's sum and its gradient
+ * when it is at most 200 KB (e.g. V = 50257 bf16), otherwise its second read
+ * comes mostly from L2 -- so one read and one write of the BT x V tensor in
+ * all, instead of flce_ce_forward's read plus flce_ce_backward's read and
+ * write.  Workspace: flce_ce_workspace_size(p, FLCE_OP_FUSED).  dlogits may
+ * be the logits array itself. */
+FLCE_API flce_status_t flce_ce_fused(const flce_ce_problem_t* p, const void* logits,
+                                     const int64_t* labels, float dloss, float* loss, float* lse,
+                                     void* dlogits, void* ws, size_t ws_bytes,
+                                     struct CUstream_st* stream);
 
 /* How flce_fused schedules its work (bf16 problems; fp32 always recomputes).
  *  FLCE_SCHEDULE_RECOMPUTE: forward pass for lse and loss, then per

@@ -5,7 +5,8 @@ the same names (the fused LM-head loss, and the cross-entropy path for callers
 that already hold the logits); ``dp`` runs it data-parallel over torch.distributed ranks;
 ``inputs`` holds the seeded synthetic workloads.
 """
-from .binding import (ce_backward, ce_forward, ce_workspace, flce_ce_backward,
+from .binding import (ce_backward, ce_forward, ce_fused, ce_workspace, flce_ce_backward,
+                      flce_ce_fused,
                       flce_ce_forward, flce_ce_problem_t, flce_ce_workspace_size,
                       make_ce_problem)
 from .binding import (FLCE_BF16, FLCE_FP32, FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_FUSED_FORWARD,

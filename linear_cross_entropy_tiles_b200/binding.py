@@ -36,7 +36,8 @@ EXPORTS = ("flce_workspace_size", "flce_forward", "flce_backward", "flce_fused",
            "flce_kernel_name", "flce_fused_noalloc", "flce_set_schedule",
            "flce_selftest_wait_timeout", "flce_count_valid", "flce_fused_global",
            "flce_ce_workspace_size", "flce_ce_forward", "flce_ce_backward",
-           "flce_selftest_approx", "flce_set_workspace_limit")
+           "flce_selftest_approx", "flce_set_workspace_limit", "flce_ce_fused",
+           "flce_vp_workspace_size", "flce_vp_forward", "flce_vp_combine", "flce_vp_backward")
 FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_RECOMPUTE, FLCE_SCHEDULE_FUSED_FORWARD = 0, 1, 2
 
 
@@ -113,11 +114,22 @@ def lib():
         L.flce_set_workspace_limit.argtypes = [ctypes.c_uint64]
         L.flce_selftest_approx.restype = ctypes.c_int
         L.flce_selftest_approx.argtypes = [p, ctypes.c_int64, p, p]
+        i64 = ctypes.c_int64
+        L.flce_vp_workspace_size.restype = ctypes.c_size_t
+        L.flce_vp_workspace_size.argtypes = [P, ctypes.c_int]
+        L.flce_vp_forward.restype = ctypes.c_int
+        L.flce_vp_forward.argtypes = [P, i64, i64, p, p, p, p, p, ctypes.c_size_t, p]
+        L.flce_vp_combine.restype = ctypes.c_int
+        L.flce_vp_combine.argtypes = [P, ctypes.c_int32, p, p, p, p, p, ctypes.c_size_t, p]
+        L.flce_vp_backward.restype = ctypes.c_int
+        L.flce_vp_backward.argtypes = [P, i64, i64, p, p, p, p, p, p, p, p, ctypes.c_size_t, p]
         C = ctypes.POINTER(flce_ce_problem_t)
         L.flce_ce_workspace_size.restype = ctypes.c_size_t
         L.flce_ce_workspace_size.argtypes = [C, ctypes.c_int]
         L.flce_ce_forward.restype = ctypes.c_int
         L.flce_ce_forward.argtypes = [C, p, p, p, p, p, ctypes.c_size_t, p]
+        L.flce_ce_fused.restype = ctypes.c_int
+        L.flce_ce_fused.argtypes = [C, p, p, ctypes.c_float, p, p, p, p, ctypes.c_size_t, p]
         L.flce_ce_backward.restype = ctypes.c_int
         L.flce_ce_backward.argtypes = [C, p, p, p, p, p, p, ctypes.c_size_t, p]
         _LIB = L
@@ -320,6 +332,53 @@ def flce_ce_backward(problem, logits, labels, lse, dloss, dlogits, ws, stream=No
                                   _stream(stream)), "flce_ce_backward")
 
 
+def flce_ce_fused(problem, logits, labels, dloss, loss, lse, dlogits, ws, stream=None):
+    """loss, lse (or None) and dlogits in one read of the logits."""
+    _check_ce(problem, logits=logits, labels=labels, lse=lse, dlogits=dlogits,
+              extra=[("loss", loss, 1, torch.float32)])
+    _check(lib().flce_ce_fused(ctypes.byref(problem), _ptr(logits), _ptr(labels), float(dloss),
+                               _ptr(loss), _ptr(lse), _ptr(dlogits), _ptr(ws), _nbytes(ws),
+                               _stream(stream)), "flce_ce_fused")
+
+
+def flce_vp_workspace_size(problem: flce_problem_t, op: int) -> int:
+    return int(lib().flce_vp_workspace_size(ctypes.byref(problem), int(op)))
+
+
+def flce_vp_forward(problem, v_offset, v_total, X, W, labels, stats, ws, stream=None):
+    """stats [BT, 3] fp32: this rank's per-row (max, sum-exp, label logit) over
+    its vocabulary slice [v_offset, v_offset + problem.V)."""
+    _check_flce(problem, X=X, W=W, labels=labels,
+                extra=[("stats", stats, 3 * problem.BT, torch.float32)])
+    _check(lib().flce_vp_forward(ctypes.byref(problem), int(v_offset), int(v_total), _ptr(X),
+                                 _ptr(W), _ptr(labels), _ptr(stats), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)), "flce_vp_forward")
+
+
+def flce_vp_combine(problem, n_ranks, stats_all, labels, loss, lse, ws, stream=None):
+    """lse and loss from all ranks' stats [n_ranks, BT, 3]; problem.V is the
+    whole vocabulary."""
+    _check_flce(problem, labels=labels, lse=lse,
+                extra=[("stats_all", stats_all, 3 * n_ranks * problem.BT, torch.float32),
+                       ("loss", loss, 1, torch.float32)])
+    _check(lib().flce_vp_combine(ctypes.byref(problem), int(n_ranks), _ptr(stats_all),
+                                 _ptr(labels), _ptr(loss), _ptr(lse), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)), "flce_vp_combine")
+
+
+def flce_vp_backward(problem, v_offset, v_total, X, W, labels, lse, dloss, dX, dW, ws,
+                     stream=None):
+    """This rank's fp32 share of dX and its rows of dW from the global lse."""
+    _check_flce(problem, X=X, W=W, labels=labels, lse=lse, dW=dW,
+                extra=[("dloss", dloss, 1, torch.float32)])
+    if isinstance(dX, torch.Tensor):
+        _check_matrix("dX", dX, problem.BT, problem.H, FLCE_FP32, problem.lddx, None)
+    _check(lib().flce_vp_backward(ctypes.byref(problem), int(v_offset), int(v_total), _ptr(X),
+                                  _ptr(W), _ptr(labels), _ptr(lse), _ptr(dloss), _ptr(dX),
+                                  _ptr(dW), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "flce_vp_backward")
+
+
 def flce_get_device_status(ws, stream=None):
     st = ctypes.c_int32(0)
     nv = ctypes.c_int64(0)
@@ -504,3 +563,18 @@ def ce_backward(logits, labels, lse, dloss, ignore_index=-100, softcap=0.0, ws=N
     ws = ce_workspace(p, FLCE_OP_BACKWARD, logits.device) if ws is None else ws
     flce_ce_backward(p, logits, labels, lse, dloss, out, ws, stream)
     return out
+
+
+def ce_fused(logits, labels, ignore_index=-100, softcap=0.0, dloss=1.0, ws=None, stream=None,
+             shift_seq_len=0, out=None, want_lse=True):
+    """Return (loss [1] fp32, lse [BT] fp32 or None, dlogits) computed by
+    flce_ce_fused; out as in ce_backward (logits itself: in place)."""
+    out = torch.empty(logits.shape, dtype=logits.dtype, device=logits.device) if out is None \
+        else out
+    p = _ce_problem_of(logits, ignore_index, softcap, shift_seq_len, out)
+    ws = ce_workspace(p, FLCE_OP_FUSED, logits.device) if ws is None else ws
+    loss = torch.empty(1, dtype=torch.float32, device=logits.device)
+    lse = torch.empty(logits.shape[0], dtype=torch.float32, device=logits.device) \
+        if want_lse else None
+    flce_ce_fused(p, logits, labels, dloss, loss, lse, out, ws, stream)
+    return loss, lse, out

@@ -114,6 +114,56 @@ __global__ void combine_kernel(const float2* __restrict__ partial, int n_tiles, 
   row_loss[row] = (labels[row] != ignore_index) ? l - target[row] : 0.f;
 }
 
+// Vocabulary parallelism, one rank's slice [v_off, v_off + n_cols) of the
+// vocabulary: per row, fold the forward GEMM's per-tile partials into the
+// slice's (largest y log2 e, sum of exp2(y log2 e - that), y at the label
+// when the label lies in the slice else 0), stats [BT][3].  Rows of another
+// rank's label and ignored rows still get the slice's max and sum.
+__global__ void vp_stats_kernel(const float2* __restrict__ partial, int n_tiles, int64_t BT,
+                                const float* __restrict__ target,
+                                const int64_t* __restrict__ labels, int64_t ignore_index,
+                                int64_t v_off, int64_t n_cols, float* __restrict__ stats,
+                                const WsHeader* hdr) {
+  const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (row >= BT || hdr->status != 0) return;
+  float m = -INFINITY;
+  for (int t = 0; t < n_tiles; ++t) m = fmaxf(m, partial[size_t(t) * BT + row].x);
+  float s = 0.f;
+  for (int t = 0; t < n_tiles; ++t) {
+    const float2 p = partial[size_t(t) * BT + row];
+    s += p.y * exp2f(p.x - m);
+  }
+  const int64_t lab = labels[row];
+  const bool here = lab != ignore_index && lab >= v_off && lab < v_off + n_cols;
+  stats[row * 3] = m;
+  stats[row * 3 + 1] = s;
+  stats[row * 3 + 2] = here ? target[row] : 0.f;
+}
+
+// Vocabulary parallelism: the ranks' slice statistics [n_ranks][BT][3],
+// combined per row in rank order: M = max of the maxima, S = sum of
+// s_r exp2(m_r - M), the target from the rank that holds it; lse and the
+// row's NLL (the mean follows in finalize_kernel).
+__global__ void vp_combine_kernel(const float* __restrict__ stats, int n_ranks, int64_t BT,
+                                  const int64_t* __restrict__ labels, int64_t ignore_index,
+                                  float* __restrict__ lse, float* __restrict__ row_loss,
+                                  const WsHeader* hdr) {
+  const int64_t row = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (row >= BT || hdr->status != 0) return;
+  const size_t rs = size_t(BT) * 3;
+  float M = -INFINITY;
+  for (int r = 0; r < n_ranks; ++r) M = fmaxf(M, stats[r * rs + row * 3]);
+  float S = 0.f, tgt = 0.f;
+  for (int r = 0; r < n_ranks; ++r) {
+    const float* st = stats + r * rs + row * 3;
+    S += st[1] * exp2f(st[0] - M);
+    tgt += st[2];
+  }
+  const float l = (M + log2f(S)) * 0.69314718055994531f;
+  lse[row] = l;
+  row_loss[row] = labels[row] != ignore_index ? l - tgt : 0.f;
+}
+
 __global__ void finalize_kernel(const float* __restrict__ row_loss, int64_t BT,
                                 const WsHeader* hdr, float* loss) {
   __shared__ double sh[1024];
@@ -151,7 +201,7 @@ __global__ void finalize_kernel(const float* __restrict__ row_loss, int64_t BT,
 // and pass 2 finishes every row of the flagged groups (blocks of unflagged
 // groups return at once); a row that was fine gets the same values again.
 constexpr int kLseQRows = 32;       // rows per block: one flag group
-constexpr int kLseQThreads = 256;   // eight warps; lane = row of the group
+constexpr int kLseQThreads = 512;   // sixteen warps; lane = row of the group
 constexpr float kRefWindow = 64.f;  // log2 units
 
 __global__ void __launch_bounds__(kLseQThreads)
@@ -175,19 +225,21 @@ __global__ void __launch_bounds__(kLseQThreads)
   const int64_t lrow = int64_t(group) * kLseQRows + lane;
   const bool in = lrow < rows;
   const int64_t row = row0 + lrow;
-  // ---- per row: max and sum of the partials; warp w takes slices w, w+8, ...
+  // ---- per row: max and sum of the partials; warp w takes slices w, w+16,
+  // ..., eight loads in flight
+  constexpr int kW = kLseQThreads / 32;
   float m = -INFINITY, sum = 0.f;
   if (in) {
     const float2* pr = partial + row;
-    for (int t = wid; t < n_parts; t += 4 * (kLseQThreads / 32)) {
-      float2 v[4];
+    for (int t = wid; t < n_parts; t += 8 * kW) {
+      float2 v[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int tt = t + u * (kLseQThreads / 32);
+      for (int u = 0; u < 8; ++u) {
+        const int tt = t + u * kW;
         v[u] = tt < n_parts ? pr[size_t(tt) * BT] : make_float2(-INFINITY, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         m = fmaxf(m, v[u].x);
         sum += v[u].y;
       }
@@ -198,7 +250,7 @@ __global__ void __launch_bounds__(kLseQThreads)
   __syncthreads();
   if (wid == 0) {
     float M = s_max[0][lane], S = s_sum[0][lane];
-    for (int w = 1; w < kLseQThreads / 32; ++w) {
+    for (int w = 1; w < kW; ++w) {
       M = fmaxf(M, s_max[w][lane]);
       S += s_sum[w][lane];
     }
@@ -239,22 +291,36 @@ __global__ void __launch_bounds__(kLseQThreads)
     if (pass == 1 && lane == 0) group_flags[group] = any != 0u;
   }
   __syncthreads();
-  // ---- Xs = bf16(f x) for the rows this pass finished: 8 columns per thread
+  // ---- Xs = bf16(f x) for the rows this pass finished: 8 columns per
+  // thread and step, two steps' loads in flight
   const int64_t vecs = H / 8;
-  for (int64_t e = tid; e < int64_t(kLseQRows) * vecs; e += kLseQThreads) {
-    const int rr = int(e / vecs);
-    const int64_t k = (e - int64_t(rr) * vecs) * 8;
-    if (!s_do[rr]) continue;
-    const int64_t lr = int64_t(group) * kLseQRows + rr;
-    const float f = s_f[rr];
-    uint4 raw = *reinterpret_cast<const uint4*>(X + (row0 + lr) * ldx + k);
-    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+  const int64_t items = int64_t(kLseQRows) * vecs;
+  for (int64_t e0 = tid; e0 < items; e0 += 2 * kLseQThreads) {
+    uint4 raw[2];
+    int rr[2];
+    int64_t k[2];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 v = __bfloat1622float2(h[q]);
-      h[q] = __floats2bfloat162_rn(v.x * f, v.y * f);
+    for (int u = 0; u < 2; ++u) {
+      const int64_t e = e0 + int64_t(u) * kLseQThreads;
+      rr[u] = e < items ? int(e / vecs) : 0;
+      k[u] = (e - int64_t(rr[u]) * vecs) * 8;
+      if (e < items && s_do[rr[u]])
+        raw[u] = *reinterpret_cast<const uint4*>(
+            X + (row0 + int64_t(group) * kLseQRows + rr[u]) * ldx + k[u]);
     }
-    *reinterpret_cast<uint4*>(Xs + lr * H + k) = raw;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t e = e0 + int64_t(u) * kLseQThreads;
+      if (e >= items || !s_do[rr[u]]) continue;
+      const float f = s_f[rr[u]];
+      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw[u]);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 v = __bfloat1622float2(h[q]);
+        h[q] = __floats2bfloat162_rn(v.x * f, v.y * f);
+      }
+      *reinterpret_cast<uint4*>(Xs + (int64_t(group) * kLseQRows + rr[u]) * H + k[u]) = raw[u];
+    }
   }
 }
 
@@ -326,6 +392,7 @@ struct SimtEpi {
   int64_t ignore_index;
   int64_t BT, H, V;
   int64_t ldx, ldw, lddx, lddw;  // row strides of X, W, dX, dW (elements)
+  int64_t label_off;             // vocabulary id of W's first row (labels are global)
   float softcap;
   // logits modes
   float2* partial;         // [ceil(V/32)][BT]
@@ -392,7 +459,7 @@ __global__ void simt_logits_kernel(const T* __restrict__ X, const T* __restrict_
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (tx == 0) ep.partial[size_t(blockIdx.x) * ep.BT + row] = make_float2(m, s);
-      if (lab == j && lab != ep.ignore_index) ep.target[row] = y;
+      if (lab == j + ep.label_off && lab != ep.ignore_index) ep.target[row] = y;
     } else {
       const long long nv = ep.hdr->n_valid;
       const bool valid = lab != ep.ignore_index && nv > 0;
@@ -401,7 +468,7 @@ __global__ void simt_logits_kernel(const T* __restrict__ X, const T* __restrict_
         const float dl = ep.dloss_dev ? *ep.dloss_dev : ep.dloss_host;
         const float p = expf(y - ep.lse[row]);
         const float d = cap ? 1.f - t * t : 1.f;
-        g = (p - (j == lab ? 1.f : 0.f)) * d * (dl / float(nv));
+        g = (p - (j + ep.label_off == lab ? 1.f : 0.f)) * d * (dl / float(nv));
       }
       if (n0 + tx < ep.ldg) ep.G[row * ep.ldg + n0 + tx] = g;
     }

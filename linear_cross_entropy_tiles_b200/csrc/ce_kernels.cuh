@@ -267,3 +267,316 @@ __global__ void __launch_bounds__(kCeThreads)
 }
 
 }  // namespace flce
+
+namespace flce {
+
+// Forward and backward in one pass over HBM, for a caller that holds the
+// logits and wants the loss and the logit gradient together: one read and
+// one write of each row instead of two reads and a write.
+//
+// ce_fused_pipe_kernel (rows up to kCeFusedRowMax bytes): a persistent block
+// per SM keeps two row buffers in shared memory.  While it works on row k
+// from one buffer -- the row's (max, sum-exp), its lse, then its gradient
+// written to global memory -- one bulk asynchronous copy brings the 16-byte
+// aligned interior of its next row into the other buffer, so the row reads
+// and the gradient writes overlap.  The few elements before the first and
+// after the last 16-byte boundary of a row go through plain loads, so every
+// access stays inside the row.  Waits on the copies are bounded: a wait that
+// gives up records FLCE_ERR_TIMEOUT, waits (bounded) for the copy still in
+// flight and returns.
+//
+// ce_fused_rows_kernel (longer rows): one block per row, the row read twice
+// (the second time mostly from L2, it was loaded moments before).  N_valid
+// must be known (labels_kernel ran first); dloss is a host value.  dZ may be
+// Z (in place).
+constexpr int kCeFusedThreads = 512;
+constexpr int kCeFusedRowMax = 112 * 1024;
+
+template <typename T, bool CAP>
+__global__ void __launch_bounds__(kCeFusedThreads, 1)
+    ce_fused_pipe_kernel(const T* Z, int64_t ld, T* dZ, int64_t ld_g, int64_t BT, int64_t V,
+                         const int64_t* __restrict__ labels, int64_t ignore_index,
+                         float softcap, float dloss, float* __restrict__ lse_out,
+                         float* __restrict__ row_loss, WsHeader* hdr, uint32_t buf_bytes,
+                         unsigned long long wait_limit_ns) {
+  using E = CeElem<T>;
+  constexpr int VE = E::kVec;
+  constexpr int kW = kCeFusedThreads / 32;
+  extern __shared__ __align__(128) uint8_t s_buf[];
+  __shared__ uint64_t full[2];
+  __shared__ float red_m[kW], red_s[kW];
+  __shared__ float s_lse2;
+  if (hdr->status != 0) return;
+  const int tid = threadIdx.x;
+  const float sc = softcap;
+  const float inv_sc = CAP ? 1.f / softcap : 0.f;
+  const long long nv = hdr->n_valid;
+  const uint64_t pol = policy_evict_first();
+  if (tid == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Row `row`'s aligned interior into buffer b (thread 0).
+  auto issue = [&](int64_t row, int b) {
+    const T* z = Z + row * ld;
+    const int64_t head = ce_head(z, V);
+    const uint32_t bytes = uint32_t(((V - head) / VE) * 16);
+    fence_proxy_async_smem();  // the buffer's earlier generic reads come first
+    if (bytes) {
+      mbar_arrive_expect_tx(&full[b], bytes);
+      bulk_load_g2s(s_buf + size_t(b) * buf_bytes, z + head, bytes, &full[b], pol);
+    } else {
+      mbar_arrive(&full[b]);
+    }
+  };
+  int64_t row = blockIdx.x;
+  if (tid == 0 && row < BT) issue(row, 0);
+  bool failed = false;
+  for (int64_t k = 0; row < BT; ++k, row += gridDim.x) {
+    const int b = int(k & 1);
+    const int64_t next = row + gridDim.x;
+    if (tid == 0 && next < BT) issue(next, b ^ 1);  // freed at the end of iteration k - 1
+    const bool got = mbar_wait_bounded(&full[b], uint32_t((k >> 1) & 1), wait_limit_ns, nullptr);
+    if (!__syncthreads_and(got)) {
+      failed = true;
+      break;
+    }
+    const T* z = Z + row * ld;
+    T* g = dZ + row * ld_g;
+    const int64_t head = ce_head(z, V);
+    const int64_t nvec = (V - head) / VE;
+    const int64_t tail0 = head + nvec * VE;
+    const uint4* sv = reinterpret_cast<const uint4*>(s_buf + size_t(b) * buf_bytes);
+    // ---- the row's max and sum
+    float m = -INFINITY, s = 0.f;
+    for (int64_t j = tid; j < head + (V - tail0); j += kCeFusedThreads) {
+      const int64_t col = j < head ? j : tail0 + (j - head);
+      ce_merge(m, s, ce_u<CAP>(E::one(z + col), sc, inv_sc), 1.f);
+    }
+    for (int64_t v0 = tid; v0 < nvec; v0 += int64_t(kCeUnroll) * kCeFusedThreads) {
+      uint4 raw[kCeUnroll];
+#pragma unroll
+      for (int u = 0; u < kCeUnroll; ++u) {
+        const int64_t v = v0 + int64_t(u) * kCeFusedThreads;
+        raw[u] = v < nvec ? sv[v] : E::neg_inf();
+      }
+      float gz = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < kCeUnroll; ++u) gz = fmaxf(gz, E::vmax(raw[u]));
+      if (gz == -INFINITY) continue;
+      const float mn = fmaxf(m, ce_u<CAP>(gz, sc, inv_sc));
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int u = 0; u < kCeUnroll; ++u) {
+        if (v0 + int64_t(u) * kCeFusedThreads >= nvec) break;
+#pragma unroll
+        for (int kk = 0; kk < VE; kk += 2) {
+          float d;
+          a0 += ex2a(fmaf(capped<CAP>(E::get(raw[u], kk), sc, inv_sc, &d), kLog2e, -mn));
+          a1 += ex2a(fmaf(capped<CAP>(E::get(raw[u], kk + 1), sc, inv_sc, &d), kLog2e, -mn));
+        }
+      }
+      s = s * ex2a(m - mn) + (a0 + a1);
+      m = mn;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+      ce_merge(m, s, m2, s2);
+    }
+    if ((tid & 31) == 0) {
+      red_m[tid >> 5] = m;
+      red_s[tid >> 5] = s;
+    }
+    __syncthreads();
+    const int64_t lab = labels[row];
+    const bool valid = lab != ignore_index;
+    if (tid == 0) {
+      float M = red_m[0], S = red_s[0];
+      for (int w = 1; w < kW; ++w) ce_merge(M, S, red_m[w], red_s[w]);
+      const float lse2 = M + log2f(S);
+      const float l = lse2 * kLn2;
+      float yt = 0.f;
+      if (valid) {
+        float d;
+        yt = capped<CAP>(E::one(z + lab), sc, inv_sc, &d);
+      }
+      if (lse_out) lse_out[row] = l;
+      row_loss[row] = valid ? l - yt : 0.f;
+      s_lse2 = lse2;
+    }
+    __syncthreads();
+    // ---- the row's gradient, from the buffer
+    const float scale = (valid && nv > 0) ? dloss / float(nv) : 0.f;
+    const float lse2 = scale != 0.f ? s_lse2 : 0.f;
+    const bool same_phase = ce_head(g, V) == head;
+    uint4* gv = reinterpret_cast<uint4*>(g + head);
+    for (int64_t j = tid; j < head + (V - tail0); j += kCeFusedThreads) {
+      const int64_t col = j < head ? j : tail0 + (j - head);
+      E::store_one(g + col, scale != 0.f ? ce_grad<CAP>(E::one(z + col), sc, inv_sc, lse2,
+                                                        scale, col == lab)
+                                         : 0.f);
+    }
+    const int64_t lab_rel = lab - head;
+    for (int64_t v = tid; v < nvec; v += kCeFusedThreads) {
+      const uint4 raw = sv[v];
+      const int64_t rel = lab_rel - v * VE;
+      float gg[VE];
+#pragma unroll
+      for (int kk = 0; kk < VE; ++kk)
+        gg[kk] = scale != 0.f
+                     ? ce_grad<CAP>(E::get(raw, kk), sc, inv_sc, lse2, scale, rel == kk)
+                     : 0.f;
+      if (same_phase) {
+        uint4 out;
+#pragma unroll
+        for (int kk = 0; kk < VE; kk += 2) E::put(out, kk, gg[kk], gg[kk + 1]);
+        __stcs(gv + v, out);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < VE; ++kk) E::store_one(g + head + v * VE + kk, gg[kk]);
+      }
+    }
+    __syncthreads();  // both buffers' readers are done before the next refill
+  }
+  if (failed && tid == 0) {
+    atomicCAS(&hdr->status, 0, kStatusTimeout);
+    // both buffers' copies may still be in flight: let them land
+    const int64_t k = (row - int64_t(blockIdx.x)) / gridDim.x;
+    mbar_wait_bounded(&full[k & 1], uint32_t((k >> 1) & 1), kDrainLimitNs, nullptr);
+    if (row + gridDim.x < BT)
+      mbar_wait_bounded(&full[(k + 1) & 1], uint32_t(((k + 1) >> 1) & 1), kDrainLimitNs,
+                        nullptr);
+  }
+}
+
+template <typename T, bool CAP>
+__global__ void __launch_bounds__(kCeFusedThreads)
+    ce_fused_rows_kernel(const T* Z, int64_t ld, T* dZ, int64_t ld_g, int64_t V,
+                    const int64_t* __restrict__ labels, int64_t ignore_index, float softcap,
+                    float dloss, float* __restrict__ lse_out, float* __restrict__ row_loss,
+                    const WsHeader* hdr) {
+  using E = CeElem<T>;
+  constexpr int VE = E::kVec;
+  constexpr int kW = kCeFusedThreads / 32;
+  __shared__ float red_m[kW], red_s[kW];
+  __shared__ float s_lse2;
+  if (hdr->status != 0) return;
+  const int64_t row = blockIdx.x;
+  const int tid = threadIdx.x;
+  const T* z = Z + row * ld;
+  T* g = dZ + row * ld_g;
+  const float sc = softcap;
+  const float inv_sc = CAP ? 1.f / softcap : 0.f;
+  const int64_t head = ce_head(z, V);
+  const int64_t nvec = (V - head) / VE;
+  const int64_t tail0 = head + nvec * VE;
+  const uint4* zv = reinterpret_cast<const uint4*>(z + head);
+  // ---- pass 1: max and sum of exp2
+  float m = -INFINITY, s = 0.f;
+  for (int64_t j = tid; j < head + (V - tail0); j += kCeFusedThreads) {
+    const int64_t col = j < head ? j : tail0 + (j - head);
+    ce_merge(m, s, ce_u<CAP>(E::one(z + col), sc, inv_sc), 1.f);
+  }
+  for (int64_t v0 = tid; v0 < nvec; v0 += int64_t(kCeUnroll) * kCeFusedThreads) {
+    uint4 raw[kCeUnroll];
+#pragma unroll
+    for (int u = 0; u < kCeUnroll; ++u) {
+      const int64_t v = v0 + int64_t(u) * kCeFusedThreads;
+      raw[u] = v < nvec ? __ldg(zv + v) : E::neg_inf();
+    }
+    float gz = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < kCeUnroll; ++u) gz = fmaxf(gz, E::vmax(raw[u]));
+    if (gz == -INFINITY) continue;
+    const float mn = fmaxf(m, ce_u<CAP>(gz, sc, inv_sc));
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int u = 0; u < kCeUnroll; ++u) {
+      if (v0 + int64_t(u) * kCeFusedThreads >= nvec) break;
+#pragma unroll
+      for (int k = 0; k < VE; k += 2) {
+        float d;
+        a0 += ex2a(fmaf(capped<CAP>(E::get(raw[u], k), sc, inv_sc, &d), kLog2e, -mn));
+        a1 += ex2a(fmaf(capped<CAP>(E::get(raw[u], k + 1), sc, inv_sc, &d), kLog2e, -mn));
+      }
+    }
+    s = s * ex2a(m - mn) + (a0 + a1);
+    m = mn;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    ce_merge(m, s, m2, s2);
+  }
+  if ((tid & 31) == 0) {
+    red_m[tid >> 5] = m;
+    red_s[tid >> 5] = s;
+  }
+  __syncthreads();
+  const int64_t lab = labels[row];
+  const bool valid = lab != ignore_index;
+  if (tid == 0) {
+    float M = red_m[0], S = red_s[0];
+    for (int w = 1; w < kW; ++w) ce_merge(M, S, red_m[w], red_s[w]);
+    const float lse2 = M + log2f(S);
+    const float l = lse2 * kLn2;
+    float yt = 0.f;
+    if (valid) {
+      float d;
+      yt = capped<CAP>(E::one(z + lab), sc, inv_sc, &d);
+    }
+    if (lse_out) lse_out[row] = l;
+    row_loss[row] = valid ? l - yt : 0.f;
+    s_lse2 = lse2;
+  }
+  __syncthreads();
+  // ---- pass 2: the gradient, reading the row again (mostly from L2)
+  const long long nv = hdr->n_valid;
+  const float scale = (valid && nv > 0) ? dloss / float(nv) : 0.f;
+  const float lse2 = scale != 0.f ? s_lse2 : 0.f;
+  const bool same_phase = ce_head(g, V) == head;
+  uint4* gv = reinterpret_cast<uint4*>(g + head);
+  for (int64_t j = tid; j < head + (V - tail0); j += kCeFusedThreads) {
+    const int64_t col = j < head ? j : tail0 + (j - head);
+    E::store_one(g + col, scale != 0.f ? ce_grad<CAP>(E::one(z + col), sc, inv_sc, lse2, scale,
+                                                      col == lab)
+                                       : 0.f);
+  }
+  const int64_t lab_rel = lab - head;
+  for (int64_t v0 = tid; v0 < nvec; v0 += int64_t(kCeUnroll) * kCeFusedThreads) {
+    uint4 raw[kCeUnroll];
+#pragma unroll
+    for (int u = 0; u < kCeUnroll; ++u) {
+      const int64_t v = v0 + int64_t(u) * kCeFusedThreads;
+      if (v < nvec) raw[u] = __ldcs(zv + v);
+    }
+#pragma unroll
+    for (int u = 0; u < kCeUnroll; ++u) {
+      const int64_t v = v0 + int64_t(u) * kCeFusedThreads;
+      if (v >= nvec) break;
+      const int64_t rel = lab_rel - v * VE;
+      float gg[VE];
+#pragma unroll
+      for (int k = 0; k < VE; ++k)
+        gg[k] = scale != 0.f
+                    ? ce_grad<CAP>(E::get(raw[u], k), sc, inv_sc, lse2, scale, rel == k)
+                    : 0.f;
+      if (same_phase) {
+        uint4 out;
+#pragma unroll
+        for (int k = 0; k < VE; k += 2) E::put(out, k, gg[k], gg[k + 1]);
+        __stcs(gv + v, out);
+      } else {
+#pragma unroll
+        for (int k = 0; k < VE; ++k) E::store_one(g + head + v * VE + k, gg[k]);
+      }
+    }
+  }
+}
+
+}  // namespace flce

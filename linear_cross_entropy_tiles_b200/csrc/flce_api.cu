@@ -45,7 +45,7 @@ enum Kind : int32_t {
   K_DWACC_GEMM, K_DX_REDUCE, K_COUNT_VALID, K_SET_NVALID, K_SHIFT_LABELS,
   // launched from flce_ce.cu (kinds fixed in internal.h)
   K_CE_FORWARD, K_CE_BACKWARD, K_CE_FUSED,
-  K_LSEQ_REPAIR, K_NUM_KINDS
+  K_LSEQ_REPAIR, K_VP_STATS, K_VP_COMBINE, K_NUM_KINDS
 };
 static_assert(int32_t(K_CE_FORWARD) == int32_t(flce_internal::kKindCeForward) &&
                   int32_t(K_CE_BACKWARD) == int32_t(flce_internal::kKindCeBackward) &&
@@ -55,7 +55,7 @@ const char* const kKindNames[K_NUM_KINDS] = {
     "labels", "lse_gemm", "lse_combine", "loss_finalize", "grad_gemm", "dx_gemm", "dw_gemm",
     "simt_lse", "simt_grad", "simt_dx", "simt_dw", "memset", "lse_q_gemm", "lse_q",
     "dw_acc_gemm", "dx_reduce", "count_valid", "set_n_valid", "shift_labels", "ce_forward",
-    "ce_backward", "ce_fused", "lse_q_repair_gemm"};
+    "ce_backward", "ce_fused", "lse_q_repair_gemm", "vp_stats", "vp_combine"};
 
 // flce_fused schedule: 0 = choose, 1 = two-pass recompute, 2 = fused-in-forward.
 std::atomic<int32_t> g_schedule{0};
@@ -95,6 +95,8 @@ struct Plan {
   int64_t BT = 0, H = 0, V = 0;
   int64_t ldx = 0, ldw = 0, lddx = 0, lddw = 0;  // row strides (elements) of X, W, dX, dW
   bool dw_f32 = false;    // bf16 inputs with an fp32 dW (the fused schedule sums into dW)
+  bool dx_f32 = false;    // bf16 inputs with an fp32 dX (vocabulary-parallel partial sums)
+  int64_t label_off = 0;  // vocabulary id of W's first row (vocabulary-parallel slice)
   size_t off_shift = 0;   // shifted labels [BT] int64 when the op shifts token ids
   bool tc = false;        // bf16 tensor-core path (else fp32 SIMT)
   int bn = 256;           // N tile of the logit GEMMs and of dX / dW
@@ -258,6 +260,7 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl) {
 }
 
 void make_plan_base(const flce_problem_t* p, int op, Plan* pl, int64_t vc_max);
+constexpr int kOpBackwardDxF32 = 32;
 
 int64_t eff_ld(int64_t ld, int64_t H) { return ld == 0 ? H : ld; }
 
@@ -287,13 +290,17 @@ void make_plan(const flce_problem_t* p, int op, Plan* pl) {
   }
 }
 
-// op FLCE_OP_FUSED + 16 (internal): the fused op on the recompute schedule.
+// op FLCE_OP_FUSED + 16 (internal): the fused op on the recompute schedule;
+// kOpBackwardDxF32: the backward writing an fp32 dX that is its own running
+// sum (no workspace for it).
 void make_plan_base(const flce_problem_t* p, int op, Plan* pl, int64_t vc_max) {
   if (op == FLCE_OP_FUSED && use_fused_forward(p)) {
     make_plan_fused_forward(p, pl);
     return;
   }
   if (op == FLCE_OP_FUSED + 16) op = FLCE_OP_FUSED;
+  const int op_in = op;
+  if (op == kOpBackwardDxF32) op = FLCE_OP_BACKWARD;
   pl->BT = p->BT;
   pl->H = p->H;
   pl->V = p->V;
@@ -343,7 +350,7 @@ void make_plan_base(const flce_problem_t* p, int op, Plan* pl, int64_t vc_max) {
   if (bwd) {
     pl->off_g = off;
     off = align256(off + rows * size_t(pl->ldg) * pl->g_elem);
-    if (pl->n_chunks > 1) {
+    if (pl->n_chunks > 1 && op_in != kOpBackwardDxF32) {
       pl->off_dxacc = off;
       off = align256(off + rows * size_t(H) * 4);
     }
@@ -543,6 +550,7 @@ TcEpi base_epi(const flce_problem_t* p, const Plan& pl, const Ptrs& q) {
   e.ld_dx = pl.lddx;
   e.ld_dw = pl.lddw;
   e.ld_acc = pl.H;
+  e.label_off = pl.label_off;
   return e;
 }
 
@@ -559,6 +567,7 @@ SimtEpi base_simt(const flce_problem_t* p, const Plan& pl, const Ptrs& q) {
   e.ldw = pl.ldw;
   e.lddx = pl.lddx;
   e.lddw = pl.lddw;
+  e.label_off = pl.label_off;
   return e;
 }
 
@@ -670,7 +679,9 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
     __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(q.ws + pl.off_g);
     CUtensorMap mx_k, mw_k, mg_k, mw_mn, mg_mn, mx_mn, mg_out, mdx_out;
     bool ok = make_map(&mg_out, G, pl.ldg, BT, pl.ldg * 2, 64, 32) &&
-              make_map(&mdx_out, q.dX, H, BT, pl.lddx * 2, 64, 32) &&
+              (pl.dx_f32 ? make_map(&mdx_out, q.dX, H, BT, pl.lddx * 4, 32, 32,
+                                    CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+                         : make_map(&mdx_out, q.dX, H, BT, pl.lddx * 2, 64, 32)) &&
               make_map(&mx_k, q.X, H, BT, pl.ldx * 2, 64, kBM) &&
               make_map(&mw_k, q.W, H, V, pl.ldw * 2, 64, b_box_rows()) &&
               make_map(&mg_k, G, pl.ldg, BT, pl.ldg * 2, 64, kBM) &&
@@ -690,7 +701,11 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
       ep.G = G;
       ep.ldg = pl.ldg;
       ep.v0 = v0;
-      ep.dx_acc = reinterpret_cast<float*>(q.ws + pl.off_dxacc);
+      // the fp32 running sum of dX over vocabulary chunks: the workspace, or
+      // the fp32 dX itself
+      ep.dx_acc = pl.dx_f32 ? static_cast<float*>(q.dX)
+                            : reinterpret_cast<float*>(q.ws + pl.off_dxacc);
+      ep.ld_acc = pl.dx_f32 ? pl.lddx : H;
       ep.dx = static_cast<__nv_bfloat16*>(q.dX);
       ep.dx_first = c == 0;
       ep.dx_last = c == pl.n_chunks - 1;
@@ -710,6 +725,7 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
       gx.b_k_off = int(v0);
       TcEpi ex = ep;
       ex.out_cols = int(H);
+      ex.out_f32 = pl.dx_f32 ? 1 : 0;
       FLCE_TRY((launch_gemm<false, true, EPI_DX>(mg_k, mw_mn, mdx_out, gx, ex, sms, st)));
       // dW_c = G_c^T X     (K = BT); the output map ends at the chunk's last row
       CUtensorMap mdw_out;
@@ -941,6 +957,8 @@ namespace flce_internal {
 void prof_before(cudaStream_t st) { ::prof_before(st); }
 void prof_after(cudaStream_t st, int32_t kind) { ::prof_after(st, kind); }
 void reset_launch_count() { t_launches = 0; }
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(); }
+int device_sm_count() { return device_sms(); }
 
 cudaError_t launch_labels(const int64_t* labels, int64_t BT, int64_t V, int64_t ignore_index,
                           void* ws, cudaStream_t st) {
@@ -1182,6 +1200,146 @@ int32_t flce_profile_stop(float* ms, int32_t* kinds, int32_t max_out) {
   g_prof.on = false;
   g_prof.cap = g_prof.n = 0;
   return ok ? out : -1;
+}
+
+// ------------------------ vocabulary parallelism ---------------------------
+
+static flce_status_t vp_check(const flce_problem_t* p, int64_t v_offset, int64_t v_total) {
+  flce_status_t s = check_problem(p);
+  if (s != FLCE_OK) return s;
+  if (p->shift_seq_len != 0) return FLCE_ERR_UNSUPPORTED;
+  if (v_offset < 0 || v_total < v_offset + p->V) return FLCE_ERR_INVALID_ARG;
+  if (v_total >= (int64_t(1) << 31)) return FLCE_ERR_UNSUPPORTED;
+  return FLCE_OK;
+}
+
+flce_status_t flce_vp_forward(const flce_problem_t* p, int64_t v_offset, int64_t v_total,
+                              const void* X, const void* W, const int64_t* labels, float* stats,
+                              void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  t_launches = 0;
+  flce_status_t s = vp_check(p, v_offset, v_total);
+  if (s != FLCE_OK) return s;
+  if ((s = check_common(p, X, W, labels, ws)) != FLCE_OK) return s;
+  if (p->BT > 0 && !stats) return FLCE_ERR_INVALID_ARG;
+  if (!aligned(stats, 4)) return FLCE_ERR_MISALIGNED;
+  Plan pl;
+  make_plan(p, FLCE_OP_FORWARD, &pl);
+  if (ws_bytes < pl.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  pl.label_off = v_offset;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  // the labels are global vocabulary ids: checked against the whole vocabulary
+  prof_before(st);
+  labels_kernel<<<1, 1024, 0, st>>>(labels, p->BT, v_total, p->ignore_index, hdr);
+  prof_after(st, K_LABELS);
+  FLCE_TRY(cudaGetLastError());
+  const int64_t BT = pl.BT, V = pl.V, H = pl.H;
+  if (BT == 0) return FLCE_OK;
+  float2* partial = reinterpret_cast<float2*>(w + pl.off_partial);
+  float* target = reinterpret_cast<float*>(w + pl.off_target);
+  Ptrs q{X, W, labels, nullptr, nullptr, nullptr, 1.f, nullptr, nullptr, w};
+  if (pl.tc) {
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, X, H, BT, pl.ldx * 2, 64, kBM)) return FLCE_ERR_CUDA;
+    if (!make_map(&mb, W, H, V, pl.ldw * 2, 64, b_box_rows())) return FLCE_ERR_CUDA;
+    TcEpi ep = base_epi(p, pl, q);
+    ep.partial = partial;
+    ep.target = target;
+    GemmArgs g{BT, V, H, true};
+    g.wide_epi = pl.part_shift == 7;
+    if (ep.softcap > 0.f)
+      FLCE_TRY((launch_gemm<false, false, EPI_LSE_CAP>(ma, mb, ma, g, ep, device_sms(), st)));
+    else
+      FLCE_TRY((launch_gemm<false, false, EPI_LSE>(ma, mb, ma, g, ep, device_sms(), st)));
+  } else {
+    SimtEpi ep = base_simt(p, pl, q);
+    ep.partial = partial;
+    ep.target = target;
+    prof_before(st);
+    simt_logits_kernel<float, 0><<<dim3(unsigned(cdiv(V, 32)), unsigned(cdiv(BT, 32))),
+                                   dim3(32, 8), 0, st>>>(static_cast<const float*>(X),
+                                                         static_cast<const float*>(W), ep);
+    prof_after(st, K_SIMT_LOGITS);
+    FLCE_TRY(cudaGetLastError());
+  }
+  prof_before(st);
+  vp_stats_kernel<<<unsigned(cdiv(BT, 256)), 256, 0, st>>>(
+      partial, int(pl.part_tiles), BT, target, labels, p->ignore_index, v_offset, V, stats, hdr);
+  prof_after(st, K_VP_STATS);
+  return cuda_status(cudaGetLastError());
+}
+
+flce_status_t flce_vp_combine(const flce_problem_t* p, int32_t n_ranks, const float* stats_all,
+                              const int64_t* labels, float* loss, float* lse, void* ws,
+                              size_t ws_bytes, struct CUstream_st* stream) {
+  t_launches = 0;
+  flce_status_t s = vp_check(p, 0, p ? p->V : 0);
+  if (s != FLCE_OK) return s;
+  if (n_ranks < 1 || !loss || !ws || (p->BT > 0 && (!stats_all || !labels || !lse)))
+    return FLCE_ERR_INVALID_ARG;
+  if (!aligned(stats_all, 4) || !aligned(labels, 8) || !aligned(loss, 4) || !aligned(lse, 4) ||
+      !aligned(ws, 256))
+    return FLCE_ERR_MISALIGNED;
+  // header and per-row losses, laid out as in the forward workspace
+  const size_t off_rowloss = kHeaderBytes + align256(size_t(p->BT) * 4);
+  if (ws_bytes < off_rowloss + align256(size_t(p->BT) * 4)) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  WsHeader* hdr = reinterpret_cast<WsHeader*>(w);
+  float* rowloss = reinterpret_cast<float*>(w + off_rowloss);
+  prof_before(st);
+  labels_kernel<<<1, 1024, 0, st>>>(labels, p->BT, p->V, p->ignore_index, hdr);
+  prof_after(st, K_LABELS);
+  FLCE_TRY(cudaGetLastError());
+  if (p->BT > 0) {
+    prof_before(st);
+    vp_combine_kernel<<<unsigned(cdiv(p->BT, 256)), 256, 0, st>>>(
+        stats_all, n_ranks, p->BT, labels, p->ignore_index, lse, rowloss, hdr);
+    prof_after(st, K_VP_COMBINE);
+    FLCE_TRY(cudaGetLastError());
+  }
+  prof_before(st);
+  finalize_kernel<<<1, 1024, 0, st>>>(rowloss, p->BT, hdr, loss);
+  prof_after(st, K_FINALIZE);
+  return cuda_status(cudaGetLastError());
+}
+
+flce_status_t flce_vp_backward(const flce_problem_t* p, int64_t v_offset, int64_t v_total,
+                               const void* X, const void* W, const int64_t* labels,
+                               const float* lse, const float* dloss, float* dX, void* dW,
+                               void* ws, size_t ws_bytes, struct CUstream_st* stream) {
+  t_launches = 0;
+  flce_status_t s = vp_check(p, v_offset, v_total);
+  if (s != FLCE_OK) return s;
+  if ((s = check_common(p, X, W, labels, ws)) != FLCE_OK) return s;
+  if (!dloss || !dW || (p->BT > 0 && (!lse || !dX))) return FLCE_ERR_INVALID_ARG;
+  if (!aligned(dX, 16) || !aligned(dW, 16) || !aligned(lse, 4) || !aligned(dloss, 4))
+    return FLCE_ERR_MISALIGNED;
+  if ((eff_ld(p->lddx, p->H) * 4) % 16 != 0) return FLCE_ERR_MISALIGNED;
+  Plan pl;
+  const bool tc = p->dtype == FLCE_BF16;
+  make_plan(p, tc ? kOpBackwardDxF32 : FLCE_OP_BACKWARD, &pl);
+  if (ws_bytes < pl.total) return FLCE_ERR_WORKSPACE_TOO_SMALL;
+  pl.dx_f32 = tc;
+  pl.label_off = v_offset;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Ptrs q{X, W, labels, nullptr, const_cast<float*>(lse), dloss, 1.f, dX, dW,
+         static_cast<uint8_t*>(ws)};
+  prof_before(st);
+  labels_kernel<<<1, 1024, 0, st>>>(labels, p->BT, v_total, p->ignore_index,
+                                    reinterpret_cast<WsHeader*>(ws));
+  prof_after(st, K_LABELS);
+  FLCE_TRY(cudaGetLastError());
+  return enqueue_backward(p, pl, q, st);
+}
+
+size_t flce_vp_workspace_size(const flce_problem_t* p, int op) {
+  if (check_problem(p) != FLCE_OK || p->shift_seq_len != 0) return 0;
+  if (op != FLCE_OP_FORWARD && op != FLCE_OP_BACKWARD) return 0;
+  Plan pl;
+  make_plan(p, op == FLCE_OP_BACKWARD && p->dtype == FLCE_BF16 ? kOpBackwardDxF32 : op, &pl);
+  return pl.total;
 }
 
 const char* flce_kernel_name(int32_t kind) {

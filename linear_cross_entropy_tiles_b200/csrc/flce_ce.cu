@@ -52,7 +52,7 @@ struct CePlan {
 void make_ce_plan(const flce_ce_problem_t* p, int op, CePlan* pl) {
   size_t off = kHeaderBytes;
   const size_t rows = size_t(p->BT);
-  if (op == FLCE_OP_FORWARD) {
+  if (op == FLCE_OP_FORWARD || op == FLCE_OP_FUSED) {
     pl->off_rowloss = off;
     off = align256(off + rows * 4);
   }
@@ -125,13 +125,57 @@ cudaError_t launch_ce_backward(const flce_ce_problem_t* p, const void* logits,
   return cudaGetLastError();
 }
 
+template <typename T, bool CAP>
+cudaError_t launch_ce_fused_t(const flce_ce_problem_t* p, const void* logits,
+                              const int64_t* labels, float dloss, float* lse, float* rowloss,
+                              void* dlogits, void* ws, cudaStream_t st) {
+  const T* Z = static_cast<const T*>(logits);
+  T* dZ = static_cast<T*>(dlogits);
+  WsHeader* hdr = static_cast<WsHeader*>(ws);
+  const int64_t ld = ld_of(p->ld, p->V), ldg = ld_of(p->ld_grad, p->V);
+  const float cap = CAP ? p->softcap : 0.f;
+  const size_t row_bytes = size_t(p->V) * sizeof(T);
+  cudaError_t e;
+  if (row_bytes <= size_t(kCeFusedRowMax)) {
+    // Two row buffers per persistent block, one block per SM.
+    const uint32_t buf = uint32_t((row_bytes + 15) / 16 * 16);
+    auto kern = ce_fused_pipe_kernel<T, CAP>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(2 * buf))) != cudaSuccess)
+      return e;
+    int grid = device_sm_count();
+    if (grid <= 0) return cudaErrorInvalidDevice;
+    if (int64_t(grid) > p->BT) grid = int(p->BT);
+    prof_before(st);
+    kern<<<unsigned(grid), kCeFusedThreads, 2 * buf, st>>>(
+        Z, ld, dZ, ldg, p->BT, p->V, labels, p->ignore_index, cap, dloss, lse, rowloss, hdr,
+        buf, wait_limit_ns());
+  } else {
+    prof_before(st);
+    ce_fused_rows_kernel<T, CAP><<<unsigned(p->BT), kCeFusedThreads, 0, st>>>(
+        Z, ld, dZ, ldg, p->V, labels, p->ignore_index, cap, dloss, lse, rowloss, hdr);
+  }
+  prof_after(st, kKindCeFused);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_ce_fused(const flce_ce_problem_t* p, const void* logits, const int64_t* labels,
+                            float dloss, float* lse, float* rowloss, void* dlogits, void* ws,
+                            cudaStream_t st) {
+  return softcap_on(p->softcap)
+             ? launch_ce_fused_t<T, true>(p, logits, labels, dloss, lse, rowloss, dlogits, ws, st)
+             : launch_ce_fused_t<T, false>(p, logits, labels, dloss, lse, rowloss, dlogits, ws,
+                                           st);
+}
+
 }  // namespace
 
 extern "C" {
 
 size_t flce_ce_workspace_size(const flce_ce_problem_t* p, int op) {
   if (check_ce(p) != FLCE_OK) return 0;
-  if (op != FLCE_OP_FORWARD && op != FLCE_OP_BACKWARD) return 0;
+  if (op != FLCE_OP_FORWARD && op != FLCE_OP_BACKWARD && op != FLCE_OP_FUSED) return 0;
   CePlan pl;
   make_ce_plan(p, op, &pl);
   return pl.total;
@@ -186,3 +230,29 @@ flce_status_t flce_ce_backward(const flce_ce_problem_t* p, const void* logits,
 }
 
 }  // extern "C"
+
+extern "C" flce_status_t flce_ce_fused(const flce_ce_problem_t* p, const void* logits,
+                                       const int64_t* labels, float dloss, float* loss,
+                                       float* lse, void* dlogits, void* ws, size_t ws_bytes,
+                                       struct CUstream_st* stream) {
+  reset_launch_count();
+  flce_status_t s = check_ce(p);
+  if (s != FLCE_OK) return s;
+  if (!loss || (p->BT > 0 && !dlogits)) return FLCE_ERR_INVALID_ARG;
+  if (!aligned(loss, 4) || !aligned(lse, 4) || !aligned(dlogits, elem_size(p->dtype)))
+    return FLCE_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CePlan pl;
+  const int64_t* lab = nullptr;
+  if ((s = prologue(p, FLCE_OP_FUSED, logits, labels, ws, ws_bytes, st, &pl, &lab)) != FLCE_OK)
+    return s;
+  float* rowloss = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_rowloss);
+  if (p->BT > 0) {
+    const cudaError_t e =
+        p->dtype == FLCE_BF16
+            ? launch_ce_fused<__nv_bfloat16>(p, logits, lab, dloss, lse, rowloss, dlogits, ws, st)
+            : launch_ce_fused<float>(p, logits, lab, dloss, lse, rowloss, dlogits, ws, st);
+    if (e != cudaSuccess) return FLCE_ERR_CUDA;
+  }
+  return launch_finalize(rowloss, p->BT, ws, loss, st) == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}

@@ -120,6 +120,9 @@ struct TcEpi {
   // and by dloss / N_valid (from n_valid, dloss_host) when scale_by_nvalid.
   const float* row_scale;
   int scale_by_nvalid;
+  // EPI_LSE / EPI_GRAD: the vocabulary id of this launch's first W row (a
+  // vocabulary-parallel rank's slice); labels are global ids.
+  int64_t label_off;
   // bf16 output tiles stored by TMA: row added to the tile row (the
   // vocabulary offset of a dW chunk) and the output tensor's column count.
   int out_row_off;
@@ -342,8 +345,9 @@ __device__ __forceinline__ void epi_lse(const TcEpi& ep, const TcShape& sh, int 
   const int64_t row = int64_t(m0) + r;
   const bool row_ok = row < sh.M;
   const int64_t lab = row_ok ? __ldg(ep.labels + row) : ep.ignore_index;
-  const int lab_col = (lab != ep.ignore_index && lab >= n0 && lab < int64_t(n0) + BN)
-                          ? int(lab - n0) : -1;
+  const int64_t labl = lab - ep.label_off;  // the label's column in this launch's W rows
+  const int lab_col = (lab != ep.ignore_index && labl >= n0 && labl < int64_t(n0) + BN)
+                          ? int(labl - n0) : -1;
   const float sc = ep.softcap;
   const float inv_sc = CAP ? 1.f / ep.softcap : 0.f;
   const int ncols = sh.N - n0;  // tile columns inside the vocabulary
@@ -407,7 +411,8 @@ __device__ __forceinline__ void epi_grad(const TcEpi& ep, const TcShape& sh, int
   // An ignored row gets lse = +inf, so every exp is 0 and G is 0 exactly.
   const float lse2 = (valid && nv > 0) ? __ldg(ep.lse + row) * kLog2e : INFINITY;
   const int64_t vbase = ep.v0 + n0;  // vocabulary index of tile column 0
-  const int lab_col = (valid && lab >= vbase && lab < vbase + BN) ? int(lab - vbase) : -1;
+  const int64_t labl = lab - ep.label_off;
+  const int lab_col = (valid && labl >= vbase && labl < vbase + BN) ? int(labl - vbase) : -1;
   const int64_t vlim = ep.V - vbase;  // tile columns >= vlim are padding
   const bool full = vlim >= c_hi * 32;
   const float sc = ep.softcap;

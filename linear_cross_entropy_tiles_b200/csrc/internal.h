@@ -20,6 +20,10 @@ void prof_before(cudaStream_t st);
 void prof_after(cudaStream_t st, int32_t kind);
 // Start counting the launches of a new entry-point call on this host thread.
 void reset_launch_count();
+// The process-wide bound on every wait inside the kernels (flce_set_wait_limit_ns).
+unsigned long long wait_limit_ns();
+// Streaming multiprocessors of the current device (0 if it cannot be read).
+int device_sm_count();
 
 // labels check + N_valid into the workspace header (status word reset).
 cudaError_t launch_labels(const int64_t* labels, int64_t BT, int64_t V, int64_t ignore_index,

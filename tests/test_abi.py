@@ -22,7 +22,7 @@ def built():
 def test_exports_every_declared_symbol():
     header = open(os.path.join(ROOT, "include", "flce.h")).read()
     declared = re.findall(r"FLCE_API\s+[\w\s\*]+?\b(flce_\w+)\s*\(", header)
-    assert len(declared) == 21
+    assert len(declared) == 26
     assert set(declared) == set(binding.EXPORTS)
     lib = binding.lib()
     for name in declared:
@@ -200,7 +200,8 @@ def test_ce_host_checks():
     fwd = flce.flce_ce_workspace_size(p, flce.FLCE_OP_FORWARD)
     bwd = flce.flce_ce_workspace_size(p, flce.FLCE_OP_BACKWARD)
     assert fwd >= 256 + 4 * 1000 and bwd == 256
-    assert flce.flce_ce_workspace_size(p, flce.FLCE_OP_FUSED) == 0
+    assert flce.flce_ce_workspace_size(p, flce.FLCE_OP_FUSED) == fwd   # flce_ce_fused
+    assert flce.flce_ce_workspace_size(p, 9) == 0
     sh = mk(1000, 50257, shift_seq_len=100)
     assert flce.flce_ce_workspace_size(sh, flce.FLCE_OP_BACKWARD) == 256 + 8192  # 256-aligned
     for bad, st in [(mk(-1, 10), 1), (mk(4, 0), 1), (mk(4, 10, ld=9), 1), (mk(4, 10, ld_grad=3), 1),
@@ -219,6 +220,12 @@ def test_ce_host_checks():
     assert L.flce_ce_forward(ctypes.byref(ok), A, A, 0, A, A, 1 << 40, None) == 1
     assert L.flce_ce_backward(ctypes.byref(ok), A, A, A, 0, A, A, 1 << 40, None) == 1
     assert L.flce_ce_backward(ctypes.byref(ok), A, A, A, A, A + 1, A, 1 << 40, None) == 3
+    # flce_ce_fused: loss required, lse optional, dlogits aligned to the element
+    assert L.flce_ce_fused(ctypes.byref(ok), A, A, 1.0, 0, A, A, A, 1 << 40, None) == 1
+    assert L.flce_ce_fused(ctypes.byref(ok), A, A, 1.0, A, A, A + 1, A, 1 << 40, None) == 3
+    assert L.flce_ce_fused(ctypes.byref(ok), A, A, 1.0, A, A, A, A, 10, None) == 4
+    for bad, st in [(mk(4, 10, ld=9), 1), (mk(4, 10, dtype=5), 2)]:
+        assert L.flce_ce_fused(ctypes.byref(bad), A, A, 1.0, A, A, A, A, 1 << 40, None) == st
 
 
 def test_binding_checks_tensors_against_the_problem():
@@ -290,3 +297,26 @@ def test_dw_fp32_problem_checks():
     for bad in (-1, 2):
         p = flce.make_problem(64, 64, 512, dw_fp32=bad)
         assert L.flce_fused(ctypes.byref(p), A, A, A, 1.0, A, A, A, A, 1 << 40, None) == 1
+
+
+def test_vocab_parallel_host_checks():
+    import ctypes
+    L = binding.lib()
+    p = flce.make_problem(64, 64, 300)
+    for op in (0, 1):
+        assert flce.binding.flce_vp_workspace_size(p, op) > 0
+    assert flce.binding.flce_vp_workspace_size(p, 2) == 0
+    sh = flce.make_problem(64, 64, 300, shift_seq_len=32)
+    assert flce.binding.flce_vp_workspace_size(sh, 0) == 0
+    for args, st in [((p, 0, 299), 1), ((p, -1, 1000), 1), ((p, 800, 1000), 1),
+                     ((sh, 0, 1000), 2), ((p, 0, 1 << 31), 2)]:
+        pr, off, tot = args
+        assert L.flce_vp_forward(ctypes.byref(pr), off, tot, A, A, A, A, A, 1 << 40, None) == st
+        assert L.flce_vp_backward(ctypes.byref(pr), off, tot, A, A, A, A, A, A, A, A, 1 << 40,
+                                  None) == st
+    assert L.flce_vp_forward(ctypes.byref(p), 0, 300, A, A, A, A + 2, A, 1 << 40, None) == 3
+    assert L.flce_vp_forward(ctypes.byref(p), 0, 300, A, A, A, A, A, 10, None) == 4
+    assert L.flce_vp_combine(ctypes.byref(p), 0, A, A, A, A, A, 1 << 40, None) == 1
+    assert L.flce_vp_combine(ctypes.byref(p), 2, A, A, A, A, A, 100, None) == 4
+    assert L.flce_vp_backward(ctypes.byref(p), 0, 300, A, A, A, A, A, A + 8, A, A, 1 << 40,
+                              None) == 3

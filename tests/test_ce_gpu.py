@@ -227,3 +227,71 @@ def test_ce_llmc_shape_full_size(cuda_device):
     row_sum = dZ.float().sum(1)
     row_abs = dZ.float().abs().sum(1)
     assert float((row_sum.abs() / row_abs.clamp_min(1e-30)).max()) <= 2e-2
+
+
+FUSED_CASES = CASES + [(8, 60000, "fp32", 3.0, 0.0, 0.0, 31),   # fp32 row > 200 KB: L2 path
+                       (16, 130001, "bf16", 3.0, 20.0, 0.1, 32)]
+
+
+@pytest.mark.parametrize("case", FUSED_CASES,
+                         ids=lambda c: "%dx%d-%s-cap%g" % (c[0], c[1], c[2], c[4]))
+def test_ce_fused_matches_oracle_and_the_two_calls(case, cuda_device):
+    """flce_ce_fused (each row read once: kept in shared memory, or re-read
+    from L2 for rows over 200 KB) against the oracle, and against the
+    forward + backward pair to fp32 rounding (their sums run in another
+    order)."""
+    BT, V, dtype, std, cap, ign, seed = case
+    Z, lab = _logits(BT, V, dtype, std, seed, ign)
+    o = _oracle(Z, lab, softcap=cap, dloss=0.75)
+    Zd, labd = Z.to(cuda_device), lab.to(cuda_device)
+    loss, lse, dZ = flce.ce_fused(Zd, labd, softcap=cap, dloss=0.75)
+    loss2, lse2 = flce.ce_forward(Zd, labd, softcap=cap)
+    dZ2 = flce.ce_backward(Zd, labd, lse2, torch.tensor([0.75], device=cuda_device), softcap=cap)
+    torch.cuda.synchronize()
+    _check(o, loss.item(), lse, dZ, dtype)
+    assert float(((lse - lse2).abs() / lse2.abs().clamp_min(1.0)).max()) <= 1e-6
+    assert rel_fro(to_np(dZ), to_np(dZ2)) <= (1e-5 if dtype == "fp32" else 4e-3)
+    ign_rows = (lab == IGN).nonzero().flatten().tolist()
+    if ign_rows:
+        assert not dZ[ign_rows].any()
+    l3, _, dZ3 = flce.ce_fused(Zd, labd, softcap=cap, dloss=0.75, want_lse=False)
+    assert l3.item() == loss.item() and torch.equal(dZ3, dZ)     # deterministic, lse optional
+
+
+@pytest.mark.parametrize("pad_out", [0, 3])
+def test_ce_fused_in_place_and_strided(pad_out, cuda_device):
+    BT, V = 130, 5003
+    Z, lab = _logits(BT, V, "bf16", 2.0, 33, 0.1)
+    Zd, labd = Z.to(cuda_device), lab.to(cuda_device)
+    ref = flce.ce_fused(Zd, labd, softcap=15.0)
+    if pad_out == 0:                       # in place
+        Zi = Zd.clone()
+        out = flce.ce_fused(Zi, labd, softcap=15.0, out=Zi)
+        assert out[2].data_ptr() == Zi.data_ptr()
+    else:                                  # output rows at another 16-byte phase
+        big = torch.full((BT, V + pad_out), 7.0, dtype=Zd.dtype, device=cuda_device)
+        out = flce.ce_fused(Zd, labd, softcap=15.0, out=big[:, :V])
+        assert bool((big[:, V:] == 7.0).all())
+    torch.cuda.synchronize()
+    assert out[0].item() == ref[0].item() and torch.equal(out[2], ref[2])
+
+
+def test_ce_fused_shift_and_llmc_full_size(cuda_device):
+    B, T, V = 3, 200, 1000
+    Z, ids = _logits(B * T, V, "bf16", 2.0, 34)
+    lab = torch.cat([ids.reshape(B, T)[:, 1:], torch.full((B, 1), IGN, dtype=ids.dtype)],
+                    1).reshape(-1)
+    loss, lse, dZ = flce.ce_fused(Z.to(cuda_device), ids.to(cuda_device), shift_seq_len=T)
+    _check(_oracle(Z, lab), loss.item(), lse, dZ, "bf16")
+    # the llm.c tensor: all rows' lse and the loss against the oracle, 512
+    # sampled gradient rows
+    w = inputs.CE_WORKLOADS["ce_llmc"]
+    Zf, labf = inputs.make_ce_workload(w, device=cuda_device)
+    loss, lse, dZ = flce.ce_fused(Zf, labf)
+    torch.cuda.synchronize()
+    Zc, labc = Zf.cpu(), labf.cpu()
+    o_all = _oracle(Zc, labc, grads=False)
+    _check(o_all, loss.item(), lse, None, "bf16")
+    R = inputs.sample_rows(w.BT, 512, seed=4)
+    o = _oracle(Zc[R], labc[R], n_valid=o_all["n_valid"])
+    assert rel_fro(to_np(dZ[R]), o["dZ"]) <= TOL["bf16"]["grad"]

@@ -180,3 +180,99 @@ def test_dw_summed_over_ranks_in_fp32(world):
     err16 = float(abs(b16[0] - ref).max()) / scale
     assert err32 <= world * 2.0 ** -23
     assert err16 >= 100 * err32 and err16 <= world * 2.0 ** -8
+
+
+def _vp_ref_stats(X, W_r, lab, v_off):
+    """fp64 torch restatement (test-only) of one rank's slice statistics."""
+    z = X @ W_r.T
+    u = z * 1.4426950408889634
+    m = u.max(dim=1).values
+    s = torch.exp2(u - m[:, None]).sum(1)
+    here = (lab >= v_off) & (lab < v_off + W_r.shape[0]) & (lab != -100)
+    idx = torch.where(here, lab - v_off, torch.zeros_like(lab))
+    tgt = torch.where(here, z[torch.arange(z.shape[0]), idx], torch.zeros_like(m))
+    return torch.stack([m, s, tgt], 1)
+
+
+def _vp_ref_combine(stats_all, lab):
+    M = stats_all[:, :, 0].max(0).values
+    S = (stats_all[:, :, 1] * torch.exp2(stats_all[:, :, 0] - M)).sum(0)
+    lse = (M + torch.log2(S)) * 0.6931471805599453
+    valid = lab != -100
+    n = int(valid.sum())
+    nll = torch.where(valid, lse - stats_all[:, :, 2].sum(0), torch.zeros_like(lse))
+    return (nll.sum() / max(n, 1)).reshape(1), lse
+
+
+def _vp_ref_backward(X, W_r, lab, v_off, lse):
+    z = X @ W_r.T
+    G = torch.exp(z - lse[:, None])
+    here = (lab >= v_off) & (lab < v_off + W_r.shape[0]) & (lab != -100)
+    rows = torch.nonzero(here).flatten()
+    G[rows, lab[rows] - v_off] -= 1.0
+    valid = lab != -100
+    n = int(valid.sum())
+    G = G * valid[:, None] / max(n, 1)
+    return G @ W_r, G.T @ X
+
+
+def _vp_worker(rank, world, port, q, X, W, lab, slices):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from linear_cross_entropy_tiles_b200 import vp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        off, n = slices[rank]
+        W_r = W[off:off + n]
+        loss, lse, dX, dW = vp.vocab_parallel_step(
+            lambda: _vp_ref_stats(X, W_r, lab, off),
+            lambda st: _vp_ref_combine(st, lab),
+            lambda l: _vp_ref_backward(X, W_r, lab, off, l))
+        q.put((rank, loss.numpy().copy(), lse.numpy().copy(), dX.numpy().copy(),
+               dW.numpy().copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_vocab_parallel_step_gloo(world):
+    """W split over the vocabulary in uneven slices: the gathered slice
+    statistics give every rank the single-process lse and loss; the summed dX
+    shares give the full dX; each rank's dW is its rows of the full dW.
+    Labels fall in every slice, one row is ignored."""
+    from linear_cross_entropy_tiles_b200 import vp
+    g = torch.Generator().manual_seed(21)
+    BT, H, V = 10, 8, 23
+    X = torch.randn(BT, H, generator=g, dtype=torch.float64)
+    W = 0.7 * torch.randn(V, H, generator=g, dtype=torch.float64)
+    lab = torch.randint(0, V, (BT,), generator=g)
+    lab[3] = -100
+    slices = vp.vp_offsets(V, world)
+    assert sum(n for _, n in slices) == V and len({n for _, n in slices}) <= 2
+    z = X @ W.T
+    lse_ref = torch.logsumexp(z, 1)
+    G = torch.softmax(z, 1)
+    valid = lab != -100
+    G[valid.nonzero().flatten(), lab[valid]] -= 1.0
+    G = G * valid[:, None] / int(valid.sum())
+    loss_ref = (lse_ref - z[torch.arange(BT), lab.clamp(min=0)])[valid].mean()
+    ctx = mp.get_context("spawn")
+    qq = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_vp_worker, args=(r, world, port, qq, X, W, lab, slices))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict((r, rest) for r, *rest in (qq.get(timeout=120) for _ in range(world)))
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    for r, (off, n) in enumerate(slices):
+        loss, lse, dX, dW = (torch.from_numpy(a) for a in got[r])
+        assert torch.allclose(loss, loss_ref.reshape(1), rtol=1e-12)
+        assert torch.allclose(lse, lse_ref, rtol=1e-12)
+        assert torch.allclose(dX, G @ W, rtol=1e-10, atol=1e-14)
+        assert torch.allclose(dW, (G.T @ X)[off:off + n], rtol=1e-10, atol=1e-14)
