@@ -307,12 +307,15 @@ FLCE_API flce_status_t flce_ce_backward(const flce_ce_problem_t* p, const void* 
 /* Forward and backward together, for a training step that holds the logits
  * (dloss by value, as flce_fused): loss (device fp32 scalar), optionally lse
  * (device fp32 [BT], or NULL) and dlogits, reading each row of the logits
- * once -- it stays in shared memory between the row's sum and its gradient
- * when it is at most 200 KB (e.g. V = 50257 bf16), otherwise its second read
- * comes mostly from L2 -- so one read and one write of the BT x V tensor in
- * all, instead of flce_ce_forward's read plus flce_ce_backward's read and
- * write.  Workspace: flce_ce_workspace_size(p, FLCE_OP_FUSED).  dlogits may
- * be the logits array itself. */
+ * from HBM once: one read and one write of the BT x V tensor in all, instead
+ * of flce_ce_forward's read plus flce_ce_backward's read and write.  Rows of
+ * at most 112 KB (V <= 57344 bf16, e.g. 50257; V <= 28672 fp32) go through
+ * one persistent block per SM that holds two rows in shared memory: the next
+ * row arrives by a bulk asynchronous copy while the current one is reduced
+ * and its gradient written.  Longer rows take one block per row, whose
+ * second read comes mostly from L2.  Workspace:
+ * flce_ce_workspace_size(p, FLCE_OP_FUSED).  dlogits may be the logits
+ * array itself. */
 FLCE_API flce_status_t flce_ce_fused(const flce_ce_problem_t* p, const void* logits,
                                      const int64_t* labels, float dloss, float* loss, float* lse,
                                      void* dlogits, void* ws, size_t ws_bytes,

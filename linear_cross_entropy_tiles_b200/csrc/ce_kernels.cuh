@@ -189,14 +189,50 @@ __global__ void __launch_bounds__(kCeThreads)
   }
 }
 
-// G for one element: (exp(y - lse) - [label]) * dy/dz * scale.
+// G for one element: (exp(y - lse) - [label]) * dy/dz * scale, evaluated as
+// p * s - [label] * s with s = dy/dz * scale -- the same operations as the
+// vector form below, so an element gets the same bits on either path.
 template <bool CAP>
 __device__ __forceinline__ float ce_grad(float z, float sc, float inv_sc, float lse2, float scale,
                                          bool is_label) {
   float d;
   const float y = capped<CAP>(z, sc, inv_sc, &d);
-  const float p = ex2a(fmaf(y, kLog2e, -lse2));
-  return (is_label ? p - 1.f : p) * (CAP ? d * scale : scale);
+  const float sd = CAP ? d * scale : scale;
+  const float g = ex2a(fmaf(y, kLog2e, -lse2)) * sd;
+  return is_label ? g - sd : g;
+}
+
+// G for the VE elements of one 16-byte vector, the one-hot term left out:
+// exp(y - lse) * dy/dz * scale.  ce_vec_label then subtracts dy/dz * scale
+// at the label, when the label falls in this vector (rel in [0, VE)): one
+// comparison per vector instead of one per element.
+template <typename T, bool CAP>
+__device__ __forceinline__ void ce_vec_grad(const uint4& raw, float sc, float inv_sc, float lse2,
+                                            float scale, float (&gg)[CeElem<T>::kVec]) {
+#pragma unroll
+  for (int k = 0; k < CeElem<T>::kVec; ++k) {
+    float d;
+    const float y = capped<CAP>(CeElem<T>::get(raw, k), sc, inv_sc, &d);
+    gg[k] = ex2a(fmaf(y, kLog2e, -lse2)) * (CAP ? d * scale : scale);
+  }
+}
+template <typename T, bool CAP>
+__device__ __forceinline__ void ce_vec_label(const uint4& raw, int rel, float sc, float inv_sc,
+                                             float scale, float (&gg)[CeElem<T>::kVec]) {
+  if (unsigned(rel) >= unsigned(CeElem<T>::kVec)) return;
+#pragma unroll
+  for (int k = 0; k < CeElem<T>::kVec; ++k)
+    if (k == rel) {
+      float d;
+      capped<CAP>(CeElem<T>::get(raw, k), sc, inv_sc, &d);
+      gg[k] -= CAP ? d * scale : scale;
+    }
+}
+// The label's position relative to the first vector of a row, as a 32-bit
+// offset (V < 2^31); a label before the vectors (in the row's head) or an
+// ignored row gives a value no vector matches.
+__device__ __forceinline__ int ce_lab_rel(int64_t lab, int64_t head, bool valid) {
+  return (valid && lab >= head) ? int(lab - head) : -1;
 }
 
 template <typename T, bool CAP>
@@ -240,27 +276,25 @@ __global__ void __launch_bounds__(kCeThreads)
     for (int64_t v = tid; v < nvec; v += kCeThreads) __stcs(gv + v, make_uint4(0u, 0u, 0u, 0u));
     return;
   }
-  const int64_t lab_rel = lab - head;  // label's position within the vector run
-  for (int64_t v0 = tid; v0 < nvec; v0 += int64_t(kCeUnroll) * kCeThreads) {
+  const int lab_rel = ce_lab_rel(lab, head, valid);  // label's position in the vector run
+  const int nv32 = int(nvec);
+  for (int v0 = tid; v0 < nv32; v0 += kCeUnroll * kCeThreads) {
     uint4 raw[kCeUnroll];
 #pragma unroll
     for (int u = 0; u < kCeUnroll; ++u) {
-      const int64_t v = v0 + int64_t(u) * kCeThreads;
-      if (v < nvec) raw[u] = __ldcs(zv + v);
+      const int v = v0 + u * kCeThreads;
+      if (v < nv32) raw[u] = __ldcs(zv + v);
     }
 #pragma unroll
     for (int u = 0; u < kCeUnroll; ++u) {
-      const int64_t v = v0 + int64_t(u) * kCeThreads;
-      if (v >= nvec) break;
-      const int64_t rel = lab_rel - v * VE;  // in [0, VE) when the label is here
+      const int v = v0 + u * kCeThreads;
+      if (v >= nv32) break;
+      float gg[VE];
+      ce_vec_grad<T, CAP>(raw[u], sc, inv_sc, lse2, scale, gg);
+      ce_vec_label<T, CAP>(raw[u], lab_rel - v * VE, sc, inv_sc, scale, gg);
       uint4 out;
 #pragma unroll
-      for (int k = 0; k < VE; k += 2) {
-        const float g0 = ce_grad<CAP>(E::get(raw[u], k), sc, inv_sc, lse2, scale, rel == k);
-        const float g1 =
-            ce_grad<CAP>(E::get(raw[u], k + 1), sc, inv_sc, lse2, scale, rel == k + 1);
-        E::put(out, k, g0, g1);
-      }
+      for (int k = 0; k < VE; k += 2) E::put(out, k, gg[k], gg[k + 1]);
       __stcs(gv + v, out);
     }
   }
@@ -274,26 +308,37 @@ namespace flce {
 // logits and wants the loss and the logit gradient together: one read and
 // one write of each row instead of two reads and a write.
 //
-// ce_fused_pipe_kernel (rows up to kCeFusedRowMax bytes): a persistent block
-// per SM keeps two row buffers in shared memory.  While it works on row k
-// from one buffer -- the row's (max, sum-exp), its lse, then its gradient
-// written to global memory -- one bulk asynchronous copy brings the 16-byte
-// aligned interior of its next row into the other buffer, so the row reads
-// and the gradient writes overlap.  The few elements before the first and
-// after the last 16-byte boundary of a row go through plain loads, so every
-// access stays inside the row.  Waits on the copies are bounded: a wait that
-// gives up records FLCE_ERR_TIMEOUT, waits (bounded) for the copy still in
-// flight and returns.
+// ce_fused_pipe_kernel (rows up to kCeFusedRowMax bytes): one persistent
+// block per SM, two row buffers in shared memory, a producer warp and
+// kCePipeWarps compute warps.
+//   producer  brings the 16-byte aligned interior of each of the block's rows
+//             into a buffer with one bulk asynchronous copy (completion
+//             counted on the buffer's `full` mbarrier) as soon as every
+//             compute warp has released the buffer (its `empty` mbarrier).
+//   compute   per row: (max, sum-exp) of the row from shared memory; one named
+//             barrier that also ANDs the warps' wait results; each warp merges
+//             the warp partials itself in the same fixed tree (no second
+//             barrier); the row's gradient written to global memory; the
+//             buffer released, and on to the next row, whose copy has
+//             usually landed by then.
+// The few elements before the first and after the last 16-byte boundary of a
+// row, and the label's logit, come from global memory through plain loads
+// issued before the wait, so every access stays inside the row.  Waits are
+// bounded: one that gives up records FLCE_ERR_TIMEOUT, the compute warps
+// leave together, and the producer waits (bounded) for its copies still in
+// flight before the block exits.
 //
 // ce_fused_rows_kernel (longer rows): one block per row, the row read twice
 // (the second time mostly from L2, it was loaded moments before).  N_valid
 // must be known (labels_kernel ran first); dloss is a host value.  dZ may be
 // Z (in place).
+constexpr int kCePipeWarps = 16;
+constexpr int kCePipeThreads = (kCePipeWarps + 1) * 32;
 constexpr int kCeFusedThreads = 512;
 constexpr int kCeFusedRowMax = 112 * 1024;
 
 template <typename T, bool CAP>
-__global__ void __launch_bounds__(kCeFusedThreads, 1)
+__global__ void __launch_bounds__(kCePipeThreads, 1)
     ce_fused_pipe_kernel(const T* Z, int64_t ld, T* dZ, int64_t ld_g, int64_t BT, int64_t V,
                          const int64_t* __restrict__ labels, int64_t ignore_index,
                          float softcap, float dloss, float* __restrict__ lse_out,
@@ -301,66 +346,96 @@ __global__ void __launch_bounds__(kCeFusedThreads, 1)
                          unsigned long long wait_limit_ns) {
   using E = CeElem<T>;
   constexpr int VE = E::kVec;
-  constexpr int kW = kCeFusedThreads / 32;
+  constexpr int kW = kCePipeWarps;
+  constexpr int kC = kW * 32;  // compute threads
   extern __shared__ __align__(128) uint8_t s_buf[];
-  __shared__ uint64_t full[2];
-  __shared__ float red_m[kW], red_s[kW];
-  __shared__ float s_lse2;
-  if (hdr->status != 0) return;
+  __shared__ uint64_t full[2], empty[2];
+  __shared__ float red_m[2][kW], red_s[2][kW];
+  __shared__ int s_skip;
   const int tid = threadIdx.x;
-  const float sc = softcap;
-  const float inv_sc = CAP ? 1.f / softcap : 0.f;
-  const long long nv = hdr->n_valid;
-  const uint64_t pol = policy_evict_first();
+  const int warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
+    // one reading of the status word for the whole block (another block may
+    // set it while this one starts)
+    s_skip = hdr->status != 0;
     mbar_init(&full[0], 1);
     mbar_init(&full[1], 1);
+    mbar_init(&empty[0], kW);
+    mbar_init(&empty[1], kW);
     fence_barrier_init();
   }
   __syncthreads();
-  // Row `row`'s aligned interior into buffer b (thread 0).
-  auto issue = [&](int64_t row, int b) {
-    const T* z = Z + row * ld;
-    const int64_t head = ce_head(z, V);
-    const uint32_t bytes = uint32_t(((V - head) / VE) * 16);
-    fence_proxy_async_smem();  // the buffer's earlier generic reads come first
-    if (bytes) {
-      mbar_arrive_expect_tx(&full[b], bytes);
-      bulk_load_g2s(s_buf + size_t(b) * buf_bytes, z + head, bytes, &full[b], pol);
-    } else {
-      mbar_arrive(&full[b]);
+  if (s_skip) return;
+  const int64_t stride = gridDim.x;
+
+  if (warp == kW) {
+    // ---- producer (one thread)
+    if (lane != 0) return;
+    const uint64_t pol = policy_evict_first();
+    bool ok = true;
+    int64_t k = 0;  // copies issued
+    for (int64_t row = blockIdx.x; row < BT; row += stride, ++k) {
+      const int b = int(k & 1);
+      // use k >> 1 of buffer b; the previous use must have been released
+      if (k >= 2 &&
+          !mbar_wait_bounded(&empty[b], uint32_t(((k >> 1) - 1) & 1), wait_limit_ns, nullptr)) {
+        ok = false;
+        break;
+      }
+      fence_proxy_async_smem();  // the released buffer's generic reads come first
+      const T* z = Z + row * ld;
+      const int64_t head = ce_head(z, V);
+      const uint32_t bytes = uint32_t(((V - head) / VE) * 16);
+      if (bytes) {
+        mbar_arrive_expect_tx(&full[b], bytes);
+        bulk_load_g2s(s_buf + size_t(b) * buf_bytes, z + head, bytes, &full[b], pol);
+      } else {
+        mbar_arrive(&full[b]);
+      }
     }
-  };
-  int64_t row = blockIdx.x;
-  if (tid == 0 && row < BT) issue(row, 0);
-  bool failed = false;
-  for (int64_t k = 0; row < BT; ++k, row += gridDim.x) {
+    if (!ok) atomicCAS(&hdr->status, 0, kStatusTimeout);
+    // the last copy into each buffer lands before the block's memory goes
+    for (int64_t j = k >= 2 ? k - 2 : 0; j < k; ++j)
+      mbar_wait_bounded(&full[j & 1], uint32_t((j >> 1) & 1), kDrainLimitNs, nullptr);
+    return;
+  }
+
+  // ---- compute warps
+  const float sc = softcap;
+  const float inv_sc = CAP ? 1.f / softcap : 0.f;
+  const long long nv = hdr->n_valid;
+  int64_t k = 0;
+  for (int64_t row = blockIdx.x; row < BT; row += stride, ++k) {
     const int b = int(k & 1);
-    const int64_t next = row + gridDim.x;
-    if (tid == 0 && next < BT) issue(next, b ^ 1);  // freed at the end of iteration k - 1
-    const bool got = mbar_wait_bounded(&full[b], uint32_t((k >> 1) & 1), wait_limit_ns, nullptr);
-    if (!__syncthreads_and(got)) {
-      failed = true;
-      break;
-    }
     const T* z = Z + row * ld;
     T* g = dZ + row * ld_g;
     const int64_t head = ce_head(z, V);
     const int64_t nvec = (V - head) / VE;
     const int64_t tail0 = head + nvec * VE;
+    const int64_t lab = labels[row];
+    const bool valid = lab != ignore_index;
+    // Plain loads, in flight during the wait: this thread's edge element (at
+    // most 2 VE - 2 per row) and, for thread 0, the label's logit.
+    int64_t edge_col = -1;
+    float edge = 0.f;
+    if (tid < head + (V - tail0)) {
+      edge_col = tid < head ? tid : tail0 + (tid - head);
+      edge = E::one(z + edge_col);
+    }
+    float zt = 0.f;
+    if (tid == 0 && valid) zt = E::one(z + lab);
+    const bool got = mbar_wait_bounded(&full[b], uint32_t((k >> 1) & 1), wait_limit_ns, nullptr);
     const uint4* sv = reinterpret_cast<const uint4*>(s_buf + size_t(b) * buf_bytes);
     // ---- the row's max and sum
     float m = -INFINITY, s = 0.f;
-    for (int64_t j = tid; j < head + (V - tail0); j += kCeFusedThreads) {
-      const int64_t col = j < head ? j : tail0 + (j - head);
-      ce_merge(m, s, ce_u<CAP>(E::one(z + col), sc, inv_sc), 1.f);
-    }
-    for (int64_t v0 = tid; v0 < nvec; v0 += int64_t(kCeUnroll) * kCeFusedThreads) {
+    if (edge_col >= 0) ce_merge(m, s, ce_u<CAP>(edge, sc, inv_sc), 1.f);
+    const int nv_here = got ? int(nvec) : 0;  // a failed wait reads nothing
+    for (int v0 = tid; v0 < nv_here; v0 += kCeUnroll * kC) {
       uint4 raw[kCeUnroll];
 #pragma unroll
       for (int u = 0; u < kCeUnroll; ++u) {
-        const int64_t v = v0 + int64_t(u) * kCeFusedThreads;
-        raw[u] = v < nvec ? sv[v] : E::neg_inf();
+        const int v = v0 + u * kC;
+        raw[u] = v < nv_here ? sv[v] : E::neg_inf();
       }
       float gz = -INFINITY;
 #pragma unroll
@@ -370,7 +445,7 @@ __global__ void __launch_bounds__(kCeFusedThreads, 1)
       float a0 = 0.f, a1 = 0.f;
 #pragma unroll
       for (int u = 0; u < kCeUnroll; ++u) {
-        if (v0 + int64_t(u) * kCeFusedThreads >= nvec) break;
+        if (v0 + u * kC >= nv_here) break;
 #pragma unroll
         for (int kk = 0; kk < VE; kk += 2) {
           float d;
@@ -387,69 +462,77 @@ __global__ void __launch_bounds__(kCeFusedThreads, 1)
       const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
       ce_merge(m, s, m2, s2);
     }
-    if ((tid & 31) == 0) {
-      red_m[tid >> 5] = m;
-      red_s[tid >> 5] = s;
+    if (lane == 0) {
+      red_m[b][warp] = m;
+      red_s[b][warp] = s;
     }
-    __syncthreads();
-    const int64_t lab = labels[row];
-    const bool valid = lab != ignore_index;
+    if (!bar_and(1, kC, got)) {  // every compute thread sees the same result
+      if (tid == 0) atomicCAS(&hdr->status, 0, kStatusTimeout);
+      return;
+    }
+    // Each warp merges the kW partials in one fixed butterfly (the merge is
+    // symmetric, so every lane and every warp gets the same bits).
+    float M = lane < kW ? red_m[b][lane] : -INFINITY;
+    float S = lane < kW ? red_s[b][lane] : 0.f;
+#pragma unroll
+    for (int o = kW / 2; o > 0; o >>= 1) {
+      const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
+      const float s2 = __shfl_xor_sync(0xffffffffu, S, o);
+      ce_merge(M, S, m2, s2);
+    }
+    M = __shfl_sync(0xffffffffu, M, 0);
+    S = __shfl_sync(0xffffffffu, S, 0);
+    const float lse2 = M + log2f(S);
     if (tid == 0) {
-      float M = red_m[0], S = red_s[0];
-      for (int w = 1; w < kW; ++w) ce_merge(M, S, red_m[w], red_s[w]);
-      const float lse2 = M + log2f(S);
       const float l = lse2 * kLn2;
       float yt = 0.f;
       if (valid) {
         float d;
-        yt = capped<CAP>(E::one(z + lab), sc, inv_sc, &d);
+        yt = capped<CAP>(zt, sc, inv_sc, &d);
       }
       if (lse_out) lse_out[row] = l;
       row_loss[row] = valid ? l - yt : 0.f;
-      s_lse2 = lse2;
     }
-    __syncthreads();
     // ---- the row's gradient, from the buffer
     const float scale = (valid && nv > 0) ? dloss / float(nv) : 0.f;
-    const float lse2 = scale != 0.f ? s_lse2 : 0.f;
+    const float l2 = scale != 0.f ? lse2 : 0.f;
+    if (edge_col >= 0)
+      E::store_one(g + edge_col, scale != 0.f ? ce_grad<CAP>(edge, sc, inv_sc, l2, scale,
+                                                             edge_col == lab)
+                                              : 0.f);
     const bool same_phase = ce_head(g, V) == head;
     uint4* gv = reinterpret_cast<uint4*>(g + head);
-    for (int64_t j = tid; j < head + (V - tail0); j += kCeFusedThreads) {
-      const int64_t col = j < head ? j : tail0 + (j - head);
-      E::store_one(g + col, scale != 0.f ? ce_grad<CAP>(E::one(z + col), sc, inv_sc, lse2,
-                                                        scale, col == lab)
-                                         : 0.f);
-    }
-    const int64_t lab_rel = lab - head;
-    for (int64_t v = tid; v < nvec; v += kCeFusedThreads) {
-      const uint4 raw = sv[v];
-      const int64_t rel = lab_rel - v * VE;
-      float gg[VE];
+    const int lab_rel = ce_lab_rel(lab, head, valid);
+    const int nv32 = int(nvec);
+    if (scale == 0.f) {  // ignored row, or no valid row at all: zeros
+      for (int v = tid; v < nv32; v += kC) {
+        if (same_phase) {
+          __stcs(gv + v, make_uint4(0u, 0u, 0u, 0u));
+        } else {
 #pragma unroll
-      for (int kk = 0; kk < VE; ++kk)
-        gg[kk] = scale != 0.f
-                     ? ce_grad<CAP>(E::get(raw, kk), sc, inv_sc, lse2, scale, rel == kk)
-                     : 0.f;
-      if (same_phase) {
-        uint4 out;
+          for (int kk = 0; kk < VE; ++kk) E::store_one(g + head + int64_t(v) * VE + kk, 0.f);
+        }
+      }
+    } else {
+#pragma unroll 2
+      for (int v = tid; v < nv32; v += kC) {
+        const uint4 raw = sv[v];
+        float gg[VE];
+        ce_vec_grad<T, CAP>(raw, sc, inv_sc, l2, scale, gg);
+        ce_vec_label<T, CAP>(raw, lab_rel - v * VE, sc, inv_sc, scale, gg);
+        if (same_phase) {
+          uint4 out;
 #pragma unroll
-        for (int kk = 0; kk < VE; kk += 2) E::put(out, kk, gg[kk], gg[kk + 1]);
-        __stcs(gv + v, out);
-      } else {
+          for (int kk = 0; kk < VE; kk += 2) E::put(out, kk, gg[kk], gg[kk + 1]);
+          __stcs(gv + v, out);
+        } else {
 #pragma unroll
-        for (int kk = 0; kk < VE; ++kk) E::store_one(g + head + v * VE + kk, gg[kk]);
+          for (int kk = 0; kk < VE; ++kk) E::store_one(g + head + int64_t(v) * VE + kk, gg[kk]);
+        }
       }
     }
-    __syncthreads();  // both buffers' readers are done before the next refill
-  }
-  if (failed && tid == 0) {
-    atomicCAS(&hdr->status, 0, kStatusTimeout);
-    // both buffers' copies may still be in flight: let them land
-    const int64_t k = (row - int64_t(blockIdx.x)) / gridDim.x;
-    mbar_wait_bounded(&full[k & 1], uint32_t((k >> 1) & 1), kDrainLimitNs, nullptr);
-    if (row + gridDim.x < BT)
-      mbar_wait_bounded(&full[(k + 1) & 1], uint32_t(((k + 1) >> 1) & 1), kDrainLimitNs,
-                        nullptr);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[b]);  // this warp is done with the buffer
   }
 }
 
@@ -547,7 +630,7 @@ __global__ void __launch_bounds__(kCeFusedThreads)
                                                       col == lab)
                                        : 0.f);
   }
-  const int64_t lab_rel = lab - head;
+  const int lab_rel = ce_lab_rel(lab, head, valid);
   for (int64_t v0 = tid; v0 < nvec; v0 += int64_t(kCeUnroll) * kCeFusedThreads) {
     uint4 raw[kCeUnroll];
 #pragma unroll
@@ -559,13 +642,14 @@ __global__ void __launch_bounds__(kCeFusedThreads)
     for (int u = 0; u < kCeUnroll; ++u) {
       const int64_t v = v0 + int64_t(u) * kCeFusedThreads;
       if (v >= nvec) break;
-      const int64_t rel = lab_rel - v * VE;
       float gg[VE];
+      if (scale != 0.f) {
+        ce_vec_grad<T, CAP>(raw[u], sc, inv_sc, lse2, scale, gg);
+        ce_vec_label<T, CAP>(raw[u], lab_rel - int(v) * VE, sc, inv_sc, scale, gg);
+      } else {
 #pragma unroll
-      for (int k = 0; k < VE; ++k)
-        gg[k] = scale != 0.f
-                    ? ce_grad<CAP>(E::get(raw[u], k), sc, inv_sc, lse2, scale, rel == k)
-                    : 0.f;
+        for (int k = 0; k < VE; ++k) gg[k] = 0.f;
+      }
       if (same_phase) {
         uint4 out;
 #pragma unroll

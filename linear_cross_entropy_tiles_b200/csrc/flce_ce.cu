@@ -137,7 +137,8 @@ cudaError_t launch_ce_fused_t(const flce_ce_problem_t* p, const void* logits,
   const size_t row_bytes = size_t(p->V) * sizeof(T);
   cudaError_t e;
   if (row_bytes <= size_t(kCeFusedRowMax)) {
-    // Two row buffers per persistent block, one block per SM.
+    // Two row buffers per persistent block, one block per SM: a producer
+    // warp and kCePipeWarps compute warps.
     const uint32_t buf = uint32_t((row_bytes + 15) / 16 * 16);
     auto kern = ce_fused_pipe_kernel<T, CAP>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -147,7 +148,7 @@ cudaError_t launch_ce_fused_t(const flce_ce_problem_t* p, const void* logits,
     if (grid <= 0) return cudaErrorInvalidDevice;
     if (int64_t(grid) > p->BT) grid = int(p->BT);
     prof_before(st);
-    kern<<<unsigned(grid), kCeFusedThreads, 2 * buf, st>>>(
+    kern<<<unsigned(grid), kCePipeThreads, 2 * buf, st>>>(
         Z, ld, dZ, ldg, p->BT, p->V, labels, p->ignore_index, cap, dloss, lse, rowloss, hdr,
         buf, wait_limit_ns());
   } else {

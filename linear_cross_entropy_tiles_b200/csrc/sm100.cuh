@@ -136,6 +136,20 @@ template <int N>
 __device__ __forceinline__ void bulk_wait_group() {
   asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
 }
+// Named barrier `id` over `n` threads (whole warps) that also ANDs a
+// predicate across them: true iff every participating thread passed true.
+__device__ __forceinline__ bool bar_and(uint32_t id, uint32_t n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(v)), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
 // Make this thread's generic-proxy shared-memory writes visible to the
 // async proxy (a following TMA store reads them).
 __device__ __forceinline__ void fence_proxy_async_smem() {

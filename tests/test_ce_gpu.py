@@ -229,15 +229,18 @@ def test_ce_llmc_shape_full_size(cuda_device):
     assert float((row_sum.abs() / row_abs.clamp_min(1e-30)).max()) <= 2e-2
 
 
-FUSED_CASES = CASES + [(8, 60000, "fp32", 3.0, 0.0, 0.0, 31),   # fp32 row > 200 KB: L2 path
-                       (16, 130001, "bf16", 3.0, 20.0, 0.1, 32)]
+FUSED_CASES = CASES + [(8, 60000, "fp32", 3.0, 0.0, 0.0, 31),   # fp32 row > 112 KB: L2 path
+                       (16, 130001, "bf16", 3.0, 20.0, 0.1, 32),
+                       # many rows per block: both row buffers reused many times
+                       (1500, 3001, "bf16", 2.0, 10.0, 0.1, 33),
+                       (2000, 700, "fp32", 3.0, 0.0, 0.05, 34)]
 
 
 @pytest.mark.parametrize("case", FUSED_CASES,
                          ids=lambda c: "%dx%d-%s-cap%g" % (c[0], c[1], c[2], c[4]))
 def test_ce_fused_matches_oracle_and_the_two_calls(case, cuda_device):
-    """flce_ce_fused (each row read once: kept in shared memory, or re-read
-    from L2 for rows over 200 KB) against the oracle, and against the
+    """flce_ce_fused (each row read once into shared memory, or re-read
+    from L2 for rows over 112 KB) against the oracle, and against the
     forward + backward pair to fp32 rounding (their sums run in another
     order)."""
     BT, V, dtype, std, cap, ign, seed = case

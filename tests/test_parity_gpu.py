@@ -29,6 +29,9 @@ CASES = [
     (70, 24, 20000, "fp32", 0.0, 0.05, 11),   # two fp32 chunks
     (200, 1096, 3000, "bf16", 0.0, 0.10, 12),  # H > 1024: four epilogue warps, ragged K
     (96, 1536, 777, "bf16", 10.0, 0.05, 13),
+    # two row chunks of the fused-in-forward schedule, the last one ragged
+    (1100, 64, 3000, "bf16", 0.0, 0.05, 14),
+    (1300, 128, 1500, "bf16", 15.0, 0.10, 15),
 ]
 
 
