@@ -548,6 +548,10 @@ def main():
                     help="steps of the second, per-launch-timed loop")
     ap.add_argument("--dw-reduce", default="fp32", choices=["fp32", "bf16"],
                     help="data parallel: dtype in which dW is written and summed over ranks")
+    ap.add_argument("--dw-slices", type=int, default=8,
+                    help="data parallel: dW handed over in this many vocabulary slices, each "
+                         "all-reduced on a side stream as soon as it is final (0: one "
+                         "all-reduce after the call)")
     ap.add_argument("--parallel", default=None, choices=["dp", "replicas"],
                     help="with several ranks: data parallel over rows (default) or "
                          "independent replicas; 'dp' on one rank runs the same step "
@@ -607,18 +611,37 @@ def main():
     stream = torch.cuda.current_stream()
 
     n_valid_buf = torch.empty(1, dtype=torch.int64, device=dev)
+    n_sl = args.dw_slices if dp_mode else 0
+    slice_bounds = flce.dw_slice_bounds(w.V, n_sl) if n_sl > 0 else []
+    slice_events = [torch.cuda.Event() for _ in slice_bounds]
+    side = torch.cuda.Stream(device=dev) if n_sl > 0 else None
 
     def compute():
         if not dp_mode:
             flce.flce_fused(p, X, W, labels, 1.0, loss, dX, dW, ws, stream)
             return
         # Data-parallel step: the count of all ranks' non-ignored labels before
-        # G is formed, then the loss shares and dW summed over the ranks.
+        # G is formed, then the loss shares and dW summed over the ranks --
+        # slice by slice on a side stream as the slices become final, or in
+        # one all-reduce after the call.
         flce.flce_count_valid(p, labels, n_valid_buf, stream)
         torch.distributed.all_reduce(n_valid_buf)
-        flce.flce_fused_global(p, X, W, labels, n_valid_buf, 1.0, loss, dX, dW, ws, stream)
+        if n_sl == 0:
+            flce.flce_fused_global(p, X, W, labels, n_valid_buf, 1.0, loss, dX, dW, ws, stream)
+            torch.distributed.all_reduce(loss)
+            torch.distributed.all_reduce(dW)
+            return
+        flce.flce_fused_global_sliced(p, X, W, labels, n_valid_buf, 1.0, loss, dX, dW, ws,
+                                      slice_events, stream)
+        works = []
+        with torch.cuda.stream(side):
+            for ev, (a, b) in zip(slice_events, slice_bounds):
+                side.wait_event(ev)
+                if b > a:
+                    works.append(torch.distributed.all_reduce(dW[a:b], async_op=True))
         torch.distributed.all_reduce(loss)
-        torch.distributed.all_reduce(dW)
+        for wk in works:
+            wk.wait()
 
     def step():
         compute()
@@ -735,7 +758,11 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-                "config": workload_config(w, world, args.parallel),
+                "config": dict(workload_config(w, world, args.parallel),
+                               **({"dw_reduce": "%s all-reduce in %s" % (
+                                   "%d overlapped vocabulary slices" % n_sl if n_sl else
+                                   "one call", "fp32" if dw32 else w.dtype)}
+                                  if dp_mode else {})),
                 "tflops": tflops, "frac_of_bf16_peak": tflops / world / peaks["bf16"],
                 "frac_of_bf16_sustained": tflops / world / peaks["bf16_sustained"],
                 "peak_basis": "%s: %.1f burst / %.1f sustained TFLOP/s dense bf16"

@@ -69,6 +69,7 @@ extern "C" {
 #endif
 
 struct CUstream_st; /* cudaStream_t is struct CUstream_st* */
+struct CUevent_st;  /* cudaEvent_t is struct CUevent_st* */
 
 #if defined(__GNUC__)
 #define FLCE_API __attribute__((visibility("default")))
@@ -174,6 +175,31 @@ FLCE_API flce_status_t flce_fused_global(const flce_problem_t* p, const void* X,
                                          const int64_t* labels, const int64_t* n_valid_global,
                                          float dloss, float* loss, void* dX, void* dW, void* ws,
                                          size_t ws_bytes, struct CUstream_st* stream);
+
+/* flce_fused_global_sliced: flce_fused_global (or flce_fused, when
+ * n_valid_global is NULL) that hands dW over in n_slices vocabulary slices,
+ * so the caller can start reducing dW over its ranks (torchtune issue #1228's
+ * data-parallel recipes: an all-reduce, or a reduce-scatter under FSDP)
+ * while the rest of dW is still being computed.  Slice s is rows
+ * [s * r, min(V, (s + 1) * r)) of dW, r = flce_dw_slice_rows(V, n_slices)
+ * (a multiple of 256; trailing slices may be empty).  slice_done[s] is a
+ * caller-created CUDA event (no timing needed); the call records it on
+ * `stream` once slice s of dW holds its final values, and writes nothing to
+ * those rows afterwards.  With the fused-in-forward schedule the last row
+ * chunk's dW GEMM runs slice by slice, each event recorded as its slice's
+ * launch ends; with the recompute schedule every event is recorded after
+ * the last launch.  1 <= n_slices <= 64, every event non-NULL (else
+ * FLCE_ERR_INVALID_ARG); otherwise as flce_fused_global. */
+FLCE_API flce_status_t flce_fused_global_sliced(const flce_problem_t* p, const void* X,
+                                                const void* W, const int64_t* labels,
+                                                const int64_t* n_valid_global, float dloss,
+                                                float* loss, void* dX, void* dW, void* ws,
+                                                size_t ws_bytes, int32_t n_slices,
+                                                struct CUevent_st* const* slice_done,
+                                                struct CUstream_st* stream);
+/* Rows of dW per slice for flce_fused_global_sliced (0 when V <= 0 or
+ * n_slices is outside [1, 64]). */
+FLCE_API int64_t flce_dw_slice_rows(int64_t V, int32_t n_slices);
 
 /* Vocabulary parallelism: W split over the vocabulary across ranks, rank r
  * holding rows [v_offset, v_offset + p->V) of a V_total-row W and all of X

@@ -12,7 +12,8 @@ from .binding import (ce_backward, ce_forward, ce_fused, ce_workspace, flce_ce_b
 from .binding import (FLCE_BF16, FLCE_FP32, FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_FUSED_FORWARD,
                       FLCE_SCHEDULE_RECOMPUTE, FLCE_OP_BACKWARD, FLCE_OP_FORWARD, FLCE_OP_FUSED,
                       FlceError, backward, count_valid, flce_backward, flce_count_valid,
-                      flce_forward, flce_fused, flce_fused_global,
+                      dw_slice_bounds, flce_dw_slice_rows, flce_forward, flce_fused,
+                      flce_fused_global, flce_fused_global_sliced,
                       flce_get_device_status, flce_kernel_name, flce_last_launch_count,
                       flce_profile_start, flce_profile_stop, flce_selftest_wait_timeout, flce_problem_t,
                       flce_set_schedule, flce_set_wait_limit_ns, flce_set_workspace_limit, flce_status_string, flce_workspace_size, forward,

@@ -37,7 +37,8 @@ EXPORTS = ("flce_workspace_size", "flce_forward", "flce_backward", "flce_fused",
            "flce_selftest_wait_timeout", "flce_count_valid", "flce_fused_global",
            "flce_ce_workspace_size", "flce_ce_forward", "flce_ce_backward",
            "flce_selftest_approx", "flce_set_workspace_limit", "flce_ce_fused",
-           "flce_vp_workspace_size", "flce_vp_forward", "flce_vp_combine", "flce_vp_backward")
+           "flce_vp_workspace_size", "flce_vp_forward", "flce_vp_combine", "flce_vp_backward",
+           "flce_fused_global_sliced", "flce_dw_slice_rows")
 FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_RECOMPUTE, FLCE_SCHEDULE_FUSED_FORWARD = 0, 1, 2
 
 
@@ -110,6 +111,12 @@ def lib():
         L.flce_fused_global.restype = ctypes.c_int
         L.flce_fused_global.argtypes = [P, p, p, p, p, ctypes.c_float, p, p, p, p,
                                         ctypes.c_size_t, p]
+        L.flce_fused_global_sliced.restype = ctypes.c_int
+        L.flce_fused_global_sliced.argtypes = [P, p, p, p, p, ctypes.c_float, p, p, p, p,
+                                               ctypes.c_size_t, ctypes.c_int32,
+                                               ctypes.POINTER(ctypes.c_void_p), p]
+        L.flce_dw_slice_rows.restype = ctypes.c_int64
+        L.flce_dw_slice_rows.argtypes = [ctypes.c_int64, ctypes.c_int32]
         L.flce_set_workspace_limit.restype = ctypes.c_uint64
         L.flce_set_workspace_limit.argtypes = [ctypes.c_uint64]
         L.flce_selftest_approx.restype = ctypes.c_int
@@ -299,6 +306,48 @@ def flce_fused_global(problem, X, W, labels, n_valid_global, dloss, loss, dX, dW
                                    _ptr(n_valid_global), float(dloss), _ptr(loss), _ptr(dX),
                                    _ptr(dW), _ptr(ws), ws.numel() * ws.element_size(),
                                    _stream(stream)), "flce_fused_global")
+
+
+def _event_handle(ev, stream):
+    """The cudaEvent_t of a torch.cuda.Event (an int passes through).  torch
+    creates an event's CUDA object on its first record, so an event never
+    recorded is recorded once on `stream` first (the call records it again)."""
+    if isinstance(ev, int):
+        return ev
+    if not ev.cuda_event:
+        ev.record(stream if stream is not None else torch.cuda.current_stream())
+    return ev.cuda_event
+
+
+def flce_fused_global_sliced(problem, X, W, labels, n_valid_global, dloss, loss, dX, dW, ws,
+                             events, stream=None):
+    """flce_fused_global (flce_fused when n_valid_global is None) recording
+    events[s] once vocabulary slice s of dW (dw_slice_bounds) is final."""
+    extra = [("loss", loss, 1, torch.float32)]
+    if n_valid_global is not None:
+        extra.append(("n_valid_global", n_valid_global, 1, torch.int64))
+    _check_flce(problem, X=X, W=W, labels=labels, dX=dX, dW=dW, extra=extra)
+    if not events:
+        raise ValueError("flce_fused_global_sliced needs at least one event")
+    handles = (ctypes.c_void_p * len(events))(*[_event_handle(e, stream) for e in events])
+    _check(lib().flce_fused_global_sliced(ctypes.byref(problem), _ptr(X), _ptr(W), _ptr(labels),
+                                          _ptr(n_valid_global), float(dloss), _ptr(loss),
+                                          _ptr(dX), _ptr(dW), _ptr(ws),
+                                          ws.numel() * ws.element_size(), len(events), handles,
+                                          _stream(stream)), "flce_fused_global_sliced")
+
+
+def flce_dw_slice_rows(V: int, n_slices: int) -> int:
+    return int(lib().flce_dw_slice_rows(int(V), int(n_slices)))
+
+
+def dw_slice_bounds(V: int, n_slices: int):
+    """[(first row, end row)] of the n_slices vocabulary slices of dW that
+    flce_fused_global_sliced hands over (trailing slices may be empty)."""
+    r = flce_dw_slice_rows(V, n_slices)
+    if r <= 0:
+        raise ValueError("need V > 0 and 1 <= n_slices <= 64")
+    return [(min(V, s * r), min(V, (s + 1) * r)) for s in range(n_slices)]
 
 
 def flce_fused_noalloc(problem, X, W, labels, dloss, loss, dX, dW, stream=None):
@@ -500,7 +549,8 @@ def backward(X, W, labels, lse, dloss, ignore_index=-100, softcap=0.0, ws=None, 
 
 
 def fused(X, W, labels, ignore_index=-100, softcap=0.0, dloss=1.0, ws=None, stream=None,
-          n_valid_global=None, shift_seq_len=0, dX=None, dW=None, dw_fp32=False):
+          n_valid_global=None, shift_seq_len=0, dX=None, dW=None, dw_fp32=False,
+          slice_events=None):
     """Return (loss [1] fp32, dX, dW) computed by flce_fused, or by
     flce_fused_global when n_valid_global (device int64 [1]) is given.
     shift_seq_len = T > 0: labels are token ids of BT/T sequences and the op
@@ -508,14 +558,19 @@ def fused(X, W, labels, ignore_index=-100, softcap=0.0, dloss=1.0, ws=None, stre
     row-strided views (e.g. a column slice of a wider tensor); dX, dW, when
     given, receive the gradients (row-strided views allowed), else dense
     tensors are allocated.  An fp32 dW (given, or dw_fp32=True) is written
-    in fp32 whatever the input type."""
+    in fp32 whatever the input type.  slice_events (torch.cuda.Event list):
+    through flce_fused_global_sliced, event s recorded once slice s of dW
+    (dw_slice_bounds(V, len(slice_events))) is final."""
     dX = torch.empty(X.shape, dtype=X.dtype, device=X.device) if dX is None else dX
     if dW is None:
         dW = torch.empty(W.shape, dtype=torch.float32 if dw_fp32 else W.dtype, device=W.device)
     p = _problem_of(X, W, ignore_index, softcap, shift_seq_len, dX, dW)
     ws = workspace(p, FLCE_OP_FUSED, X.device) if ws is None else ws
     loss = torch.empty(1, dtype=torch.float32, device=X.device)
-    if n_valid_global is None:
+    if slice_events:
+        flce_fused_global_sliced(p, X, W, labels, n_valid_global, dloss, loss, dX, dW, ws,
+                                 slice_events, stream)
+    elif n_valid_global is None:
         flce_fused(p, X, W, labels, dloss, loss, dX, dW, ws, stream)
     else:
         flce_fused_global(p, X, W, labels, n_valid_global, dloss, loss, dX, dW, ws, stream)

@@ -87,6 +87,8 @@ constexpr size_t kHeaderBytes = 256;
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+// Most vocabulary slices dW may be handed over in (flce_fused_global_sliced).
+constexpr int32_t kMaxDwSlices = 64;
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // ------------------------------- planning ----------------------------------
@@ -535,7 +537,23 @@ struct Ptrs {
   void* dW;
   uint8_t* ws;
   const int64_t* n_valid_global = nullptr;  // device count over all ranks, or null
+  // dW handed over in vocabulary slices: event s recorded once rows
+  // [s * slice_rows, (s + 1) * slice_rows) of dW are final (none: 0 / null)
+  int32_t n_slices = 0;
+  cudaEvent_t* slice_done = nullptr;
 };
+
+// Rows of dW per slice when dW is handed over in n vocabulary slices: the
+// slices are [s * r, min(V, (s + 1) * r)) with r a multiple of 256 (whole
+// GEMM tiles), so some trailing slices may be empty.
+int64_t dw_slice_rows(int64_t V, int32_t n) { return round_up(cdiv(V, int64_t(n)), 256); }
+
+// Record every slice's event at once (paths whose dW is final only at the end).
+flce_status_t record_all_slices(const Ptrs& q, cudaStream_t st) {
+  for (int32_t s = 0; s < q.n_slices; ++s)
+    if (cudaEventRecord(q.slice_done[s], st) != cudaSuccess) return FLCE_ERR_CUDA;
+  return FLCE_OK;
+}
 
 TcEpi base_epi(const flce_problem_t* p, const Plan& pl, const Ptrs& q) {
   TcEpi e{};
@@ -913,9 +931,38 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     if (!ew.dx_last && !make_map(&macc, ew.dx_acc, H, V, size_t(ew.ld_acc) * 4, 32, 32,
                                  CU_TENSOR_MAP_DATA_TYPE_FLOAT32))
       return FLCE_ERR_CUDA;
-    GemmArgs gw{V, H, rows, false};
-    FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, ew.dx_last ? mdw_out : macc, gw,
-                                              ew, sms, st, K_DWACC_GEMM)));
+    if (ew.dx_last && q.n_slices > 0) {
+      // The last chunk's dW GEMM in vocabulary slices, each slice's rows of
+      // dW final when its launch ends: the same GEMM with M = the slice's
+      // rows, the A operand (P^T) offset to the slice's first column and the
+      // outputs' base pointers to its first row.
+      const int64_t vs = dw_slice_rows(V, q.n_slices);
+      for (int32_t sl = 0; sl < q.n_slices; ++sl) {
+        const int64_t v0 = int64_t(sl) * vs;
+        if (v0 < V) {
+          const int64_t vn = (V - v0) < vs ? (V - v0) : vs;
+          TcEpi es = ew;
+          es.dx_acc = ew.dx_acc + v0 * ew.ld_acc;
+          if (!pl.dw_f32) es.dx = ew.dx + v0 * pl.lddw;
+          CUtensorMap mo;
+          const bool ok = pl.dw_f32
+                              ? make_map(&mo, static_cast<float*>(q.dW) + v0 * pl.lddw, H, vn,
+                                         pl.lddw * 4, 32, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32)
+                              : make_map(&mo, static_cast<__nv_bfloat16*>(q.dW) + v0 * pl.lddw,
+                                         H, vn, pl.lddw * 2, 64, 32);
+          if (!ok) return FLCE_ERR_CUDA;
+          GemmArgs gs{vn, H, rows, false};
+          gs.a_mn_off = int(v0);
+          FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, mo, gs, es, sms, st,
+                                                    K_DWACC_GEMM)));
+        }
+        if (cudaEventRecord(q.slice_done[sl], st) != cudaSuccess) return FLCE_ERR_CUDA;
+      }
+    } else {
+      GemmArgs gw{V, H, rows, false};
+      FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, ew.dx_last ? mdw_out : macc, gw,
+                                                ew, sms, st, K_DWACC_GEMM)));
+    }
   }
   prof_before(st);
   finalize_kernel<<<1, 1024, 0, st>>>(rowloss, BT, hdr, q.loss);
@@ -1045,10 +1092,15 @@ flce_status_t flce_backward(const flce_problem_t* p, const void* X, const void* 
 static flce_status_t fused_impl(const flce_problem_t* p, const void* X, const void* W,
                          const int64_t* labels, const int64_t* n_valid_global, float dloss,
                          float* loss, void* dX, void* dW, void* ws, size_t ws_bytes,
-                         struct CUstream_st* stream) {
+                         struct CUstream_st* stream, int32_t n_slices = 0,
+                         struct CUevent_st* const* slice_done = nullptr) {
   t_launches = 0;
   flce_status_t s = check_problem(p);
   if (s != FLCE_OK) return s;
+  if (n_slices < 0 || n_slices > kMaxDwSlices || (n_slices > 0 && !slice_done))
+    return FLCE_ERR_INVALID_ARG;
+  for (int32_t i = 0; i < n_slices; ++i)
+    if (!slice_done[i]) return FLCE_ERR_INVALID_ARG;
   if ((s = check_common(p, X, W, labels, ws)) != FLCE_OK) return s;
   if (!loss || !dW || (p->BT > 0 && !dX)) return FLCE_ERR_INVALID_ARG;
   if (!aligned(loss, 4) || !aligned(dX, 16) || !aligned(dW, 16)) return FLCE_ERR_MISALIGNED;
@@ -1059,12 +1111,17 @@ static flce_status_t fused_impl(const flce_problem_t* p, const void* X, const vo
   uint8_t* w = static_cast<uint8_t*>(ws);
   Ptrs q{X, W, labels, loss, reinterpret_cast<float*>(w + pl.off_lse), nullptr, dloss, dX, dW,
          w, n_valid_global};
+  q.n_slices = n_slices;
+  q.slice_done = reinterpret_cast<cudaEvent_t*>(const_cast<CUevent_st**>(slice_done));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if ((s = enqueue_shift(p, pl, &q, st)) != FLCE_OK) return s;
   if ((s = enqueue_labels(p, q, st)) != FLCE_OK) return s;
   if (pl.fused_fwd) return enqueue_fused_forward(p, pl, q, st);
   if ((s = enqueue_forward(p, pl, q, st)) != FLCE_OK) return s;
-  return enqueue_backward(p, pl, q, st);
+  if ((s = enqueue_backward(p, pl, q, st)) != FLCE_OK) return s;
+  // the recompute schedule writes each vocabulary chunk's dW rows once, but
+  // the slices are handed over together at the end
+  return record_all_slices(q, st);
 }
 
 flce_status_t flce_fused(const flce_problem_t* p, const void* X, const void* W,
@@ -1079,6 +1136,22 @@ flce_status_t flce_fused_global(const flce_problem_t* p, const void* X, const vo
                                 size_t ws_bytes, struct CUstream_st* stream) {
   if (!n_valid_global) return FLCE_ERR_INVALID_ARG;
   return fused_impl(p, X, W, labels, n_valid_global, dloss, loss, dX, dW, ws, ws_bytes, stream);
+}
+
+flce_status_t flce_fused_global_sliced(const flce_problem_t* p, const void* X, const void* W,
+                                       const int64_t* labels, const int64_t* n_valid_global,
+                                       float dloss, float* loss, void* dX, void* dW, void* ws,
+                                       size_t ws_bytes, int32_t n_slices,
+                                       struct CUevent_st* const* slice_done,
+                                       struct CUstream_st* stream) {
+  if (n_slices < 1) return FLCE_ERR_INVALID_ARG;
+  return fused_impl(p, X, W, labels, n_valid_global, dloss, loss, dX, dW, ws, ws_bytes, stream,
+                    n_slices, slice_done);
+}
+
+int64_t flce_dw_slice_rows(int64_t V, int32_t n_slices) {
+  if (V <= 0 || n_slices < 1 || n_slices > kMaxDwSlices) return 0;
+  return dw_slice_rows(V, n_slices);
 }
 
 flce_status_t flce_count_valid(const flce_problem_t* p, const int64_t* labels, int64_t* n_valid,

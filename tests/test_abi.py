@@ -22,7 +22,7 @@ def built():
 def test_exports_every_declared_symbol():
     header = open(os.path.join(ROOT, "include", "flce.h")).read()
     declared = re.findall(r"FLCE_API\s+[\w\s\*]+?\b(flce_\w+)\s*\(", header)
-    assert len(declared) == 26
+    assert len(declared) == 28
     assert set(declared) == set(binding.EXPORTS)
     lib = binding.lib()
     for name in declared:
@@ -320,3 +320,27 @@ def test_vocab_parallel_host_checks():
     assert L.flce_vp_combine(ctypes.byref(p), 2, A, A, A, A, A, 100, None) == 4
     assert L.flce_vp_backward(ctypes.byref(p), 0, 300, A, A, A, A, A, A + 8, A, A, 1 << 40,
                               None) == 3
+
+
+def test_sliced_call_host_checks():
+    """flce_fused_global_sliced rejects a slice count outside [1, 64] and a
+    NULL event before any CUDA call; flce_dw_slice_rows gives whole 256-row
+    tiles that cover V."""
+    import ctypes
+    L = binding.lib()
+    p = flce.make_problem(64, 64, 512)
+    ev = (ctypes.c_void_p * 2)(A, A)
+    args = (ctypes.byref(p), A, A, A, None, 1.0, A, A, A, A, 1 << 40)
+    assert L.flce_fused_global_sliced(*args, 0, ev, None) == 1
+    assert L.flce_fused_global_sliced(*args, 65, ev, None) == 1
+    assert L.flce_fused_global_sliced(*args, 2, None, None) == 1
+    assert L.flce_fused_global_sliced(*args, 2, (ctypes.c_void_p * 2)(A, None), None) == 1
+    assert flce.flce_dw_slice_rows(128256, 8) == 16128
+    assert flce.flce_dw_slice_rows(1000, 8) == 256
+    assert flce.flce_dw_slice_rows(0, 4) == 0 and flce.flce_dw_slice_rows(10, 0) == 0
+    assert flce.flce_dw_slice_rows(10, 65) == 0
+    for V, n in ((128256, 8), (256000, 3), (50257, 64), (1, 1), (300, 2)):
+        b = flce.dw_slice_bounds(V, n)
+        assert len(b) == n and b[0][0] == 0 and b[-1][1] == V
+        assert all(x1 == y0 for (_, x1), (y0, _) in zip(b, b[1:]))
+        assert all((y - x) % 256 == 0 or y == V for x, y in b)

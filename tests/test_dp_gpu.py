@@ -100,3 +100,61 @@ def test_fused_dp_one_rank_nccl_equals_fused(cuda_device):
         assert dW16.dtype == torch.bfloat16 and torch.equal(dW16, ref[2])
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("sched", ["recompute", "fused_fwd"])
+@pytest.mark.parametrize("n_slices,dw_fp32", [(1, False), (4, False), (8, False), (3, True)])
+def test_sliced_dW_equals_unsliced(sched, n_slices, dw_fp32, cuda_device):
+    """flce_fused_global_sliced: the last row chunk's dW GEMM in vocabulary
+    slices of whole 256-row tiles computes the same tiles in the same order,
+    so loss, dX and dW equal flce_fused's bit for bit (V = 3000 in 8 slices
+    of 512 rows leaves two empty); every slice's event is recorded; the
+    fused-in-forward schedule launches one dW GEMM per non-empty slice in
+    its last row chunk, and dW may be a row-strided view."""
+    BT, H, V, cap = 1100, 128, 3000, 5.0
+    X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.05, 0.1, 65, device=cuda_device)
+    prev = flce.flce_set_schedule({"recompute": flce.FLCE_SCHEDULE_RECOMPUTE,
+                                   "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD}[sched])
+    try:
+        ref = flce.fused(X, W, lab, softcap=cap, dloss=0.5, dw_fp32=dw_fp32)
+        events = [torch.cuda.Event() for _ in range(n_slices)]
+        dt = torch.float32 if dw_fp32 else torch.bfloat16
+        big = torch.full((V, H + 8), 3.0, dtype=dt, device=cuda_device)
+        flce.flce_profile_start(256)
+        out = flce.fused(X, W, lab, softcap=cap, dloss=0.5, dW=big[:, :H], slice_events=events)
+        names = [k for k, _ in flce.flce_profile_stop()]
+    finally:
+        flce.flce_set_schedule(prev)
+    torch.cuda.synchronize()
+    assert all(e.query() for e in events)
+    assert torch.equal(out[0], ref[0]) and torch.equal(out[1], ref[1])
+    assert torch.equal(out[2], ref[2]) and bool((big[:, H:] == 3.0).all())
+    bounds = flce.dw_slice_bounds(V, n_slices)
+    assert bounds[0][0] == 0 and bounds[-1][1] == V
+    assert all(b0 == a1 for (_, b0), (a1, _) in zip(bounds, bounds[1:]))
+    if sched == "fused_fwd":
+        nonempty = sum(b > a for a, b in bounds)
+        assert names.count("dw_acc_gemm") == names.count("lse_q_gemm") - 1 + nonempty
+
+
+def test_fused_dp_sliced_and_sharded_one_rank_nccl(cuda_device):
+    """dp.fused_dp reducing dW slice by slice on a side stream (all-reduce),
+    or onto one rank per slice (reduce-scatter), over a one-rank NCCL group:
+    equal to flce_fused bit for bit; the shard of the only rank is all of dW."""
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(_free_port()))
+    dist.init_process_group("nccl", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=cuda_device)
+    try:
+        X, W, lab = inputs.make_inputs(1100, 128, 3000, "bf16", 1.0, 0.05, 0.05, 66,
+                                       device=cuda_device)
+        ref = flce.fused(X, W, lab, dw_fp32=True)
+        loss, dX, dW, n = dp.fused_dp(X, W, lab, dw_slices=3)
+        l2, dX2, dW2, _ = dp.fused_dp(X, W, lab, dw_shard=True)
+        torch.cuda.synchronize()
+        assert int(n.item()) == int((lab != -100).sum().item())
+        for lo, dx, dw in ((loss, dX, dW), (l2, dX2, dW2)):
+            assert torch.equal(lo, ref[0]) and torch.equal(dx, ref[1])
+            assert dw.shape == ref[2].shape and torch.equal(dw, ref[2])
+    finally:
+        dist.destroy_process_group()

@@ -128,6 +128,72 @@ def test_data_parallel_step_gloo_world2():
             assert torch.allclose(dX, ref_dX[rows], rtol=1e-12, atol=1e-14)
 
 
+def _sliced_worker(rank, world, port, q, shards, bounds, shard):
+    import datetime
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from linear_cross_entropy_tiles_b200 import dp
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        X, W, lab = shards[rank]
+
+        def compute(n, events):
+            assert events is None  # CPU tensors: final when compute returns
+            return _ref_step(X, W, lab, n)
+
+        loss, dX, dW, n = dp.data_parallel_step_sliced(
+            lambda: (lab != -100).sum().reshape(1).to(torch.int64), compute, bounds,
+            shard=shard)
+        q.put((rank, loss.numpy().copy(), dX.numpy().copy(), dW.numpy().copy(), int(n.item())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,shard", [(2, False), (3, False), (2, True), (3, True)])
+def test_sliced_dW_exchange_gloo(world, shard):
+    """The overlapped exchange of flce_fused_global_sliced's dW: slices of
+    whole 256-row tiles (here 4-row pieces of a 37-row dW, trailing slices
+    empty), each all-reduced, or reduced onto its rank (reduce-scatter):
+    every rank gets the summed dW, or exactly its own rows of it."""
+    g = torch.Generator().manual_seed(11)
+    H, V, BT = 8, 37, 14
+    X = torch.randn(BT, H, generator=g, dtype=torch.float64)
+    W = 0.3 * torch.randn(V, H, generator=g, dtype=torch.float64)
+    lab = torch.randint(0, V, (BT,), generator=g)
+    lab[[1, 9]] = -100
+    cuts = [0, 4, 9, BT][:world] + [BT]
+    shards = [(X[cuts[r]:cuts[r + 1]], W, lab[cuts[r]:cuts[r + 1]]) for r in range(world)]
+    n_all = torch.tensor([int((lab != -100).sum())])
+    ref_loss, ref_dX, ref_dW = _ref_step(X, W, lab, n_all)
+    if shard:
+        r = 16  # rows per slice; the third rank's slice is empty when world = 3
+        bounds = [(min(V, s * r), min(V, (s + 1) * r)) for s in range(world)]
+    else:
+        bounds = [(0, 12), (12, 24), (24, 37), (37, 37)]
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sliced_worker, args=(r, world, port, q, shards, bounds, shard))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = dict((r, rest) for r, *rest in (q.get(timeout=120) for _ in range(world)))
+    for p in procs:
+        p.join(timeout=120)
+    assert all(p.exitcode == 0 for p in procs)
+    for r in range(world):
+        loss, dX, dW, n = got[r]
+        assert n == int(n_all.item())
+        assert torch.allclose(torch.from_numpy(loss), ref_loss, rtol=1e-12, atol=1e-14)
+        assert torch.allclose(torch.from_numpy(dX), ref_dX[cuts[r]:cuts[r + 1]], rtol=1e-12,
+                              atol=1e-14)
+        want = ref_dW[bounds[r][0]:bounds[r][1]] if shard else ref_dW
+        assert tuple(dW.shape) == tuple(want.shape)
+        assert torch.allclose(torch.from_numpy(dW), want, rtol=1e-12, atol=1e-14)
+
+
 def _dw_reduce_worker(rank, world, port, q, shares):
     import datetime
     import sys
