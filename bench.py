@@ -528,6 +528,9 @@ def main():
     ap.add_argument("--workload", default="llama3_8b")
     ap.add_argument("--bt", type=int, default=0,
                     help="override BT of the workload (small cases for profiling)")
+    ap.add_argument("--v", type=int, default=0,
+                    help="override V of an LM-head workload (small cases for profiling "
+                         "that keep the full-size K of every GEMM)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--schedule", default="auto", choices=["auto", "recompute", "fused_fwd"],
                     help="flce_fused schedule (auto: fused-in-forward for BT >= 512)")
@@ -588,15 +591,16 @@ def main():
     build.build()
     dev = torch.device("cuda", torch.cuda.current_device())
     w = inputs.WORKLOADS[args.workload]
-    if args.bt:
+    if args.bt or args.v:
         import dataclasses
-        w = dataclasses.replace(w, BT=args.bt)
+        w = dataclasses.replace(w, BT=args.bt or w.BT, V=args.v or w.V)
     if args.parallel == "dp" and world > 1:
         import dataclasses
         w = dataclasses.replace(w, seed=w.seed + 1000 * rank)  # each rank its own rows
     X, W, labels = inputs.make_workload(w, device=dev)
     if args.parallel == "dp" and world > 1:
-        W = inputs.make_workload(inputs.WORKLOADS[args.workload], device=dev, BT=1)[1]
+        W = inputs.make_workload(dataclasses.replace(w, seed=inputs.WORKLOADS[args.workload].seed),
+                                 device=dev, BT=1)[1]  # the same W on every rank
     flce.flce_set_schedule({"auto": 0, "recompute": 1, "fused_fwd": 2}[args.schedule])
     dp_mode = args.parallel == "dp"
     # Data parallel: each rank writes its dW share in fp32 and the ranks sum
@@ -694,7 +698,7 @@ def main():
                 "peak_kind": peak_kind, "profiled_steps": prof_steps,
                 "flops_per_launch": flops_per_step.get(dom, 0.0) / launches_dom,
                 "avg_launch_ms": dom_time_per_step / launches_dom,
-                "traffic": traffic_of(dom, args.workload, args.schedule, args.bt),
+                "traffic": traffic_of(dom, args.workload, args.schedule, args.bt or args.v),
                 "shares": {k: round(v[0] / total_prof, 4) for k, v in sorted(by_kind.items())}}
 
     # End to end through the public API with host buffers.  Per step, the
