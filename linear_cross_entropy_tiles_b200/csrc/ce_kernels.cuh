@@ -332,7 +332,11 @@ namespace flce {
 // (the second time mostly from L2, it was loaded moments before).  N_valid
 // must be known (labels_kernel ran first); dloss is a host value.  dZ may be
 // Z (in place).
-constexpr int kCePipeWarps = 16;
+#ifndef FLCE_CE_PIPE_WARPS
+#define FLCE_CE_PIPE_WARPS 16
+#endif
+constexpr int kCePipeWarps = FLCE_CE_PIPE_WARPS;
+static_assert(kCePipeWarps >= 1 && kCePipeWarps <= 31, "compute warps of one block, plus one");
 constexpr int kCePipeThreads = (kCePipeWarps + 1) * 32;
 constexpr int kCeFusedThreads = 512;
 constexpr int kCeFusedRowMax = 112 * 1024;
@@ -470,12 +474,15 @@ __global__ void __launch_bounds__(kCePipeThreads, 1)
       if (tid == 0) atomicCAS(&hdr->status, 0, kStatusTimeout);
       return;
     }
-    // Each warp merges the kW partials in one fixed butterfly (the merge is
-    // symmetric, so every lane and every warp gets the same bits).
+    // Each warp merges the kW partials in one fixed butterfly (lanes past kW
+    // hold the identity; the merge is symmetric, so every lane and every
+    // warp gets the same bits): over kW lanes when kW is a power of two,
+    // else over all 32.
+    constexpr int kSpan = (kW & (kW - 1)) == 0 ? kW : 32;
     float M = lane < kW ? red_m[b][lane] : -INFINITY;
     float S = lane < kW ? red_s[b][lane] : 0.f;
 #pragma unroll
-    for (int o = kW / 2; o > 0; o >>= 1) {
+    for (int o = kSpan / 2; o > 0; o >>= 1) {
       const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
       const float s2 = __shfl_xor_sync(0xffffffffu, S, o);
       ce_merge(M, S, m2, s2);
