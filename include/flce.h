@@ -18,7 +18,7 @@
  *                                   issue #1228)
  *   G      = (softmax(y) - onehot(label)) * dy/dz * dloss / N_valid, rows with
  *            ignored labels zero; the softmax is recomputed from X, W and the
- *            saved lse ("it can be recompute from softmax_input", PR #126348),
+ *            saved lse (PR #126348, point b: the softmax is rebuilt, not saved),
  *            or, in flce_fused for BT >= 512, rebuilt from the bf16
  *            exp(y - m) the forward kept for one chunk of rows at a time
  *   dX     = G W,    dW = G^T X
@@ -125,8 +125,8 @@ FLCE_API size_t flce_workspace_size(const flce_problem_t* p, int op);
 
 /* Forward: loss (device fp32 scalar) and lse (device fp32 [BT], the per-row
  * log-sum-exp that flce_backward needs).  Steps 1-3 of the PR #126348
- * summary with the target-logit gather in place of step 4 ("only a small
- * slice of the softmax_output tensor is need to compute NLLLoss"). */
+ * summary with the target-logit gather in place of step 4 (the PR's point
+ * a: the NLL needs one entry of each softmax row, not the whole tensor). */
 FLCE_API flce_status_t flce_forward(const flce_problem_t* p, const void* X, const void* W,
                            const int64_t* labels, float* loss, float* lse, void* ws,
                            size_t ws_bytes, struct CUstream_st* stream);

@@ -11,8 +11,8 @@
 //             -> dX (+)= G_c W_c   (fp32 running sum, bf16 on the last chunk)
 //             -> dW_c  = G_c^T X   (complete per chunk: its K is all of BT)
 // The logits of the backward are recomputed from X, W and the saved lse
-// instead of being stored (PyTorch PR #126348: "it can be recompute from
-// softmax_input" and the max/sum tensors).
+// instead of being stored (PyTorch PR #126348, point b: the softmax is rebuilt
+// from softmax_input and the small per-row statistics, never saved).
 #include <atomic>
 #include <cmath>
 #include <cstdint>

@@ -11,9 +11,9 @@
 //   warps 2..5  epilogue: tcgen05.ld of 32 to 128 columns at a time, one
 //               thread per accumulator row (TMEM lane), then one of
 //     EPI_LSE  -- per-row online max / sum of exp over the tile's columns and
-//                 the target-logit gather ("load softmax_input to compute max
-//                 per row", "... sum per row", PyTorch PR #126348 steps 2-3,
-//                 done on the tile in registers instead of re-reading HBM);
+//                 the target-logit gather (the row max and row sum passes,
+//                 steps 2 and 3 of PyTorch PR #126348's summary, done on the
+//                 tile in registers instead of re-reading HBM);
 //     EPI_GRAD -- G = (exp(y - lse) - onehot) * dy/dz * dloss / N, rounded to
 //                 bf16 into the chunk buffer (the softmax recomputed from the
 //                 saved row statistics, PR #126348 point b);
