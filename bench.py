@@ -540,7 +540,8 @@ def main():
     ap.add_argument("--ce-mode", default="separate", choices=["separate", "fused"],
                     help="ce_* workloads: flce_ce_forward + flce_ce_backward (the PR's two "
                          "passes), or flce_ce_fused (one read of the logits)")
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=0,
+                    help="timed end-to-end steps (0: as many as --steps)")
     ap.add_argument("--e2e-copies", default="data", choices=["data", "all"],
                     help="e2e host copies per step: the step's data in and the loss out "
                          "(default), or also W in and the gradients out")
@@ -561,6 +562,8 @@ def main():
                          "independent replicas; 'dp' on one rank runs the same step "
                          "over a one-rank group")
     args = ap.parse_args()
+    if args.e2e_steps <= 0:
+        args.e2e_steps = args.steps
     world_env = int(os.environ.get("WORLD_SIZE", "1"))
     if args.parallel is None:
         args.parallel = "dp" if world_env > 1 else "replicas"
@@ -621,7 +624,7 @@ def main():
     slice_events = [torch.cuda.Event() for _ in slice_bounds]
     side = torch.cuda.Stream(device=dev) if n_sl > 0 else None
 
-    def compute():
+    def compute(X=X, labels=labels):
         if not dp_mode:
             flce.flce_fused(p, X, W, labels, 1.0, loss, dX, dW, ws, stream)
             return
@@ -718,25 +721,52 @@ def main():
         dXh = torch.empty_like(dX, device="cpu").pin_memory() if copy_all else None
         dWh = torch.empty_like(dW, device="cpu").pin_memory() if copy_all else None
 
-        def e2e_step():
-            X.copy_(Xh, non_blocking=True)
-            if copy_all:
-                W.copy_(Wh, non_blocking=True)
-            labels.copy_(Lh, non_blocking=True)
-            compute()
-            lossh.copy_(loss, non_blocking=True)
-            if copy_all:
-                dXh.copy_(dX, non_blocking=True)
-                dWh.copy_(dW, non_blocking=True)
+        # The step's data arrive as a training loop's loader delivers them:
+        # step i's X and labels are copied into one of two device buffers on
+        # a copy stream while step i - 1 computes (the first copy inside the
+        # timed region too).  With --e2e-copies all every copy stays on the
+        # compute stream, in order.
+        bufs = [(X, labels), (torch.empty_like(X), torch.empty_like(labels))]
+        cstream = torch.cuda.Stream(device=dev)
+        ready = [torch.cuda.Event(), torch.cuda.Event()]
+        free = [torch.cuda.Event(), torch.cuda.Event()]
 
-        e2e_step()
+        def issue_copy(i):
+            xb, lb = bufs[i % 2]
+            cstream.wait_event(free[i % 2])  # step i - 2 is done with this buffer
+            with torch.cuda.stream(cstream):
+                xb.copy_(Xh, non_blocking=True)
+                lb.copy_(Lh, non_blocking=True)
+                ready[i % 2].record(cstream)
+
+        def e2e_steps(n):
+            if copy_all:
+                for _ in range(n):
+                    X.copy_(Xh, non_blocking=True)
+                    W.copy_(Wh, non_blocking=True)
+                    labels.copy_(Lh, non_blocking=True)
+                    compute()
+                    lossh.copy_(loss, non_blocking=True)
+                    dXh.copy_(dX, non_blocking=True)
+                    dWh.copy_(dW, non_blocking=True)
+                return
+            cstream.wait_stream(stream)  # the first copy starts inside the timed region
+            issue_copy(0)
+            for i in range(n):
+                if i + 1 < n:
+                    issue_copy(i + 1)
+                stream.wait_event(ready[i % 2])
+                compute(*bufs[i % 2])
+                free[i % 2].record(stream)
+                lossh.copy_(loss, non_blocking=True)
+
+        e2e_steps(2)
         torch.cuda.synchronize()
         barrier(world)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
+        e2e_steps(args.e2e_steps)
         e1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
@@ -748,8 +778,10 @@ def main():
             d2h += dXh.numel() * dXh.element_size() + dWh.numel() * dWh.element_size()
         e2e = {"value": world * w.BT / (ems / 1e3), "unit": "tokens/s", "ms_per_step": ems,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "copies": ("X, labels, W in; loss, dX, dW out" if copy_all else
-                          "X, labels in; loss out (W resident, dX and dW stay on the device)"),
+               "copies": ("X, labels, W in; loss, dX, dW out, in order on the compute stream"
+                          if copy_all else
+                          "X, labels in (on a copy stream, one step ahead, two device "
+                          "buffers); loss out (W resident, dX and dW stay on the device)"),
                "api": ("linear_cross_entropy_tiles_b200 flce_count_valid + flce_fused_global "
                        "(C ABI) + torch.distributed all-reduces" if dp_mode else
                        "linear_cross_entropy_tiles_b200.flce_fused (C ABI)")}
