@@ -344,3 +344,19 @@ def test_sliced_call_host_checks():
         assert len(b) == n and b[0][0] == 0 and b[-1][1] == V
         assert all(x1 == y0 for (_, x1), (y0, _) in zip(b, b[1:]))
         assert all((y - x) % 256 == 0 or y == V for x, y in b)
+
+
+def test_recorded_traffic_and_profiles_describe_this_build():
+    """bench.py's DRAM-traffic table and the ncu summaries under profiles/
+    name the hash of the kernel sources they were captured from; both must
+    describe the sources as they stand (a kernel change needs new captures)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    h = bench.csrc_sha16()
+    assert all(t["csrc_sha16"] == h for t in bench.TRAFFIC.values())
+    prof = os.path.join(ROOT, "profiles")
+    names = sorted(n for n in os.listdir(prof) if n.endswith(".md"))
+    assert names
+    for n in names:
+        assert h in open(os.path.join(prof, n)).read(), n
