@@ -103,6 +103,21 @@ __device__ __forceinline__ void ce_merge(float& m, float& s, float m2, float s2)
   m = mn;
 }
 
+// Combine the 32 lanes' (max, sum of exp2(u - max)) pairs: the max by an
+// xor butterfly, each lane's sum rescaled to it (one exp2), the sums by a
+// second butterfly.  Every step is symmetric in its two operands, so all
+// lanes end with the same bits.  An empty lane is (-inf, 0).
+__device__ __forceinline__ void ce_warp_combine(float& m, float& s) {
+  float M = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float S = (m == -INFINITY) ? 0.f : s * ex2a(m - M);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+  m = M;
+  s = S;
+}
+
 template <typename T, bool CAP>
 __global__ void __launch_bounds__(kCeThreads)
     ce_forward_kernel(const T* __restrict__ Z, int64_t ld, int64_t V,
@@ -460,12 +475,10 @@ __global__ void __launch_bounds__(kCePipeThreads, 1)
       s = s * ex2a(m - mn) + (a0 + a1);
       m = mn;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
-      const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-      ce_merge(m, s, m2, s2);
-    }
+    // The warp's (max, sum): the largest max by one butterfly, every lane's
+    // sum rescaled to it once, then summed by a second butterfly (each step
+    // symmetric, so every lane holds the same bits).
+    ce_warp_combine(m, s);
     if (lane == 0) {
       red_m[b][warp] = m;
       red_s[b][warp] = s;
@@ -474,21 +487,11 @@ __global__ void __launch_bounds__(kCePipeThreads, 1)
       if (tid == 0) atomicCAS(&hdr->status, 0, kStatusTimeout);
       return;
     }
-    // Each warp merges the kW partials in one fixed butterfly (lanes past kW
-    // hold the identity; the merge is symmetric, so every lane and every
-    // warp gets the same bits): over kW lanes when kW is a power of two,
-    // else over all 32.
-    constexpr int kSpan = (kW & (kW - 1)) == 0 ? kW : 32;
+    // Each warp combines the kW partials the same way (lanes past kW hold
+    // the identity), so every lane and every warp gets the same bits.
     float M = lane < kW ? red_m[b][lane] : -INFINITY;
     float S = lane < kW ? red_s[b][lane] : 0.f;
-#pragma unroll
-    for (int o = kSpan / 2; o > 0; o >>= 1) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, M, o);
-      const float s2 = __shfl_xor_sync(0xffffffffu, S, o);
-      ce_merge(M, S, m2, s2);
-    }
-    M = __shfl_sync(0xffffffffu, M, 0);
-    S = __shfl_sync(0xffffffffu, S, 0);
+    ce_warp_combine(M, S);
     const float lse2 = M + log2f(S);
     if (tid == 0) {
       const float l = lse2 * kLn2;
