@@ -54,16 +54,16 @@ METRIC = ("FLCE fwd+bwd tokens/s and TFLOP/s (% of B200 BF16 peak); peak extra H
 # are reported as null for any other build or workload.
 TRAFFIC = {
     ("llama3_8b", "auto"): {
-        "csrc_sha16": "d88b86de8e1ecda8",
-        "bytes_per_launch": {"lse_q_gemm": 2.4445e9, "dx_gemm": 6.195e9, "dw_acc_gemm": 4.981e9,
+        "csrc_sha16": "8dea23cbe5ebac1f",
+        "bytes_per_launch": {"lse_q_gemm": 2.3815e9, "dx_gemm": 5.5945e9, "dw_acc_gemm": 5.0345e9,
                              "lse_q": 0.0255e9}},
     ("gpt2_small", "auto"): {
-        "csrc_sha16": "d88b86de8e1ecda8",
-        "bytes_per_launch": {"lse_q_gemm": 0.888e9, "dx_gemm": 1.054e9,
+        "csrc_sha16": "8dea23cbe5ebac1f",
+        "bytes_per_launch": {"lse_q_gemm": 0.890e9, "dx_gemm": 1.0545e9,
                              "dw_acc_gemm": 1.183e9}},
     ("ce_llmc", "auto"): {
-        "csrc_sha16": "d88b86de8e1ecda8",
-        "bytes_per_launch": {"ce_forward": 3.297e9, "ce_backward": 6.541e9,
+        "csrc_sha16": "8dea23cbe5ebac1f",
+        "bytes_per_launch": {"ce_forward": 3.298e9, "ce_backward": 6.542e9,
                              "ce_fused": 6.531e9}},
 }
 

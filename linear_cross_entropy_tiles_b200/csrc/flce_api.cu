@@ -223,6 +223,13 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl) {
   if (cmax < 128) cmax = 128;
   int64_t n = cdiv(BT, cmax);
   if (BT > 128 && n < 2) n = 2;
+  // ... and chunks whose X rows (the forward GEMM's reused operand) stay
+  // within 46 MiB, so they stay in L2 beside the streaming W and q: on the
+  // Llama-3 shape a 67 MB chunk made the forward GEMM 7 % slower, and on
+  // ragged BT from 12k to 34k rows chunks of 4224-5632 rows (this cap) beat
+  // the memory cap's 6300-6900 by 1-3 %.
+  const int64_t x_rows = (int64_t(46) << 20) / (2 * H) / 128 * 128;
+  if (x_rows >= 128 && cdiv(BT, x_rows) > n) n = cdiv(BT, x_rows);
   pl->Cb = round_up(cdiv(BT, n), 128);
   pl->n_row_chunks = cdiv(BT, pl->Cb);
   size_t off = kHeaderBytes;
