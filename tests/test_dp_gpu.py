@@ -158,3 +158,28 @@ def test_fused_dp_sliced_and_sharded_one_rank_nccl(cuda_device):
             assert dw.shape == ref[2].shape and torch.equal(dw, ref[2])
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("capped", [False, True])
+def test_sliced_dW_with_shift_softcap_and_workspace_cap(capped, cuda_device):
+    """The sliced hand-over composes with the in-op label shift and the
+    softcap, and with a workspace cap that sends the automatic schedule to
+    the recompute plan (whose events are all recorded after its last
+    launch): equal to the unsliced call bit for bit in each case."""
+    B, T, H, V, cap = 5, 240, 128, 3000, 20.0
+    X, W, ids = inputs.make_inputs(B * T, H, V, "bf16", 1.0, 0.05, 0.0, 67, device=cuda_device)
+    p = flce.make_problem(B * T, H, V, torch.bfloat16, softcap=cap, shift_seq_len=T)
+    prev = flce.flce_set_workspace_limit(1 << 20 if capped else 0)
+    try:
+        ref = flce.fused(X, W, ids, softcap=cap, shift_seq_len=T)
+        events = [torch.cuda.Event() for _ in range(5)]
+        out = flce.fused(X, W, ids, softcap=cap, shift_seq_len=T, slice_events=events)
+        ws_size = flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
+    finally:
+        flce.flce_set_workspace_limit(prev)
+    torch.cuda.synchronize()
+    assert all(e.query() for e in events)
+    for a, b in zip(out, ref):
+        assert torch.equal(a, b)
+    if capped:
+        assert ws_size < 64 << 20  # the capped plan is the recompute schedule
