@@ -313,6 +313,10 @@ def workload_config(w, world, parallel="replicas"):
 
 
 SCHEDULE = ["auto"]
+# --schedule names: flce_set_schedule values (the fused-in-forward schedule
+# with dW passes by the library's rule, one per row chunk, or one over all rows)
+SCHEDULES = {"auto": 0, "recompute": 1, "fused_fwd": 2, "fused_fwd_dw_per_chunk": 3,
+             "fused_fwd_dw_once": 4}
 
 
 def run_ragged(args, world, rank):
@@ -322,7 +326,7 @@ def run_ragged(args, world, rank):
     import linear_cross_entropy_tiles_b200 as flce
     from linear_cross_entropy_tiles_b200 import build, inputs
     build.build()
-    flce.flce_set_schedule({"auto": 0, "recompute": 1, "fused_fwd": 2}[args.schedule])
+    flce.flce_set_schedule(SCHEDULES[args.schedule])
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     bts = inputs.ragged_bt_list()
@@ -533,7 +537,7 @@ def main():
                     help="override V of an LM-head workload (small cases for profiling "
                          "that keep the full-size K of every GEMM)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--schedule", default="auto", choices=["auto", "recompute", "fused_fwd"],
+    ap.add_argument("--schedule", default="auto", choices=list(SCHEDULES),
                     help="flce_fused schedule (auto: fused-in-forward for BT >= 512)")
     ap.add_argument("--cpu-rows", type=int, default=8)
     ap.add_argument("--ce-cpu-rows", type=int, default=8192)
@@ -605,7 +609,7 @@ def main():
     if args.parallel == "dp" and world > 1:
         W = inputs.make_workload(dataclasses.replace(w, seed=inputs.WORKLOADS[args.workload].seed),
                                  device=dev, BT=1)[1]  # the same W on every rank
-    flce.flce_set_schedule({"auto": 0, "recompute": 1, "fused_fwd": 2}[args.schedule])
+    flce.flce_set_schedule(SCHEDULES[args.schedule])
     dp_mode = args.parallel == "dp"
     # Data parallel: each rank writes its dW share in fp32 and the ranks sum
     # it in fp32 (--dw-reduce bf16: bf16 shares summed in bf16).

@@ -351,15 +351,24 @@ FLCE_API flce_status_t flce_ce_fused(const flce_ce_problem_t* p, const void* log
  *  FLCE_SCHEDULE_RECOMPUTE: forward pass for lse and loss, then per
  *    vocabulary chunk recompute the logits, form G and run dX and dW
  *    (8*BT*H*V FLOP; workspace < one BT x V bf16 tensor by far).
- *  FLCE_SCHEDULE_FUSED_FORWARD: per row chunk keep p = exp(y - tile max)
- *    of the forward GEMM (bf16), turn it into G once the chunk's lse is
- *    known, run dX for the chunk and add the chunk's dW in fp32
- *    (6*BT*H*V FLOP; workspace ~1 GiB of p plus an fp32 V x H sum).
+ *  FLCE_SCHEDULE_FUSED_FORWARD: per row chunk (at least two; at most
+ *    1 GiB of q, 2 GiB when an fp32 V x H array exceeds 1 GiB, and 46 MiB
+ *    of X rows each) the forward GEMM keeps q = exp(y) dy/dz in bf16 against
+ *    one exponent reference per row, the chunk's lse and row factors follow,
+ *    and dX for the chunk is q W scaled per row (6*BT*H*V FLOP).  dW is
+ *    one GEMM over every row when the q of all rows is no larger than one
+ *    chunk's q plus an fp32 V x H array (workspace: that q, about one bf16
+ *    BT x V tensor), else one GEMM per chunk summed in an fp32 V x H array
+ *    (workspace: a chunk's q plus that array, unless dW is fp32).
+ *  FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK, FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE:
+ *    the same with dW always per chunk, or always over every row.
  *  FLCE_SCHEDULE_AUTO: fused-in-forward when BT >= 512, else recompute. */
 typedef enum {
   FLCE_SCHEDULE_AUTO = 0,
   FLCE_SCHEDULE_RECOMPUTE = 1,
-  FLCE_SCHEDULE_FUSED_FORWARD = 2
+  FLCE_SCHEDULE_FUSED_FORWARD = 2,
+  FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK = 3,
+  FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE = 4
 } flce_schedule_t;
 
 /* Set the process-wide flce_fused schedule (also used by
@@ -370,7 +379,8 @@ FLCE_API int32_t flce_set_schedule(int32_t schedule);
 /* Process-wide cap, in bytes, on the workspace flce_fused plans under
  * FLCE_SCHEDULE_AUTO (0 = none, the default; also used by
  * flce_workspace_size for FLCE_OP_FUSED).  Under the cap AUTO takes the
- * fused-in-forward schedule only when its workspace fits, else the
+ * fused-in-forward schedule only when its workspace fits (first with its
+ * own choice of dW passes, then with one dW GEMM per chunk), else the
  * recompute schedule with its vocabulary chunk narrowed (down to 256
  * columns) until the workspace fits; when nothing fits it plans the
  * smallest recompute workspace.  A cap of one bf16 BT x V tensor (2*BT*V
