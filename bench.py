@@ -54,17 +54,17 @@ METRIC = ("FLCE fwd+bwd tokens/s and TFLOP/s (% of B200 BF16 peak); peak extra H
 # are reported as null for any other build or workload.
 TRAFFIC = {
     ("llama3_8b", "auto"): {
-        "csrc_sha16": "8dea23cbe5ebac1f",
-        "bytes_per_launch": {"lse_q_gemm": 2.3815e9, "dx_gemm": 5.5945e9, "dw_acc_gemm": 5.0345e9,
+        "csrc_sha16": "fbcd890a5973ffee",
+        "bytes_per_launch": {"lse_q_gemm": 2.3438e9, "dx_gemm": 5.6258e9, "dw_acc_gemm": 8.4876e9,
                              "lse_q": 0.0255e9}},
     ("gpt2_small", "auto"): {
-        "csrc_sha16": "8dea23cbe5ebac1f",
-        "bytes_per_launch": {"lse_q_gemm": 0.890e9, "dx_gemm": 1.0545e9,
-                             "dw_acc_gemm": 1.183e9}},
+        "csrc_sha16": "fbcd890a5973ffee",
+        "bytes_per_launch": {"lse_q_gemm": 0.888e9, "dx_gemm": 1.055e9,
+                             "dw_acc_gemm": 1.182e9}},
     ("ce_llmc", "auto"): {
-        "csrc_sha16": "8dea23cbe5ebac1f",
-        "bytes_per_launch": {"ce_forward": 3.298e9, "ce_backward": 6.542e9,
-                             "ce_fused": 6.531e9}},
+        "csrc_sha16": "fbcd890a5973ffee",
+        "bytes_per_launch": {"ce_forward": 3.299e9, "ce_backward": 6.5415e9,
+                             "ce_fused": 6.530e9}},
 }
 
 
@@ -278,6 +278,54 @@ def profile_kinds(step, n_steps, launches_per_step):
         k[0] += t
         k[1] += 1
     return by_kind
+
+
+def cublas_floor(w, X, W, compute, stream, rounds):
+    """The same shape's three dense GEMMs in cuBLAS (torch.mm): logits
+    X W^T into a bf16 BT x V buffer, then G W and G^T X from it -- the
+    6 BT H V FLOP of the fused call with no softmax, no exponentials and no
+    per-row work -- timed in alternation with the fused call on the same
+    stream (rounds of a few calls each), so both see the same clocks.  V is
+    padded to a multiple of 64 for cuBLAS (rows of 16-byte multiples keep
+    it on its tensor-core kernels).  Medians over the rounds, ms per call."""
+    Vp = (w.V + 63) // 64 * 64
+    Wp = torch.zeros(Vp, w.H, dtype=W.dtype, device=W.device)
+    Wp[:w.V].copy_(W)
+    G = torch.empty(w.BT, Vp, dtype=X.dtype, device=X.device)
+    dXc, dWc = torch.empty_like(X), torch.empty_like(Wp)
+    parts = {"forward": lambda: torch.mm(X, Wp.t(), out=G),
+             "dx": lambda: torch.mm(G, Wp, out=dXc),
+             "dw": lambda: torch.mm(G.t(), X, out=dWc)}
+
+    def three():
+        for f in parts.values():
+            f()
+
+    def timed(f, n):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            f()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+    n = 10 if w.BT * w.H * w.V < 8e12 else 6
+    for f in (compute, three, compute, three):
+        f()
+    torch.cuda.synchronize()
+    rows = []
+    for _ in range(rounds):
+        r = {"ours": timed(compute, n), "cublas": timed(three, n)}
+        r.update({k: timed(f, n) for k, f in parts.items()})
+        rows.append(r)
+    med = {k: sorted(r[k] for r in rows)[len(rows) // 2] for k in rows[0]}
+    del G, dXc, dWc, Wp
+    torch.cuda.empty_cache()
+    return {"ms": med["cublas"], "ours_ms_interleaved": med["ours"],
+            "per_gemm_ms": {k: med[k] for k in parts}, "rounds": rounds, "calls_per_round": n,
+            "v_padded": Vp, "api": "torch.mm (cuBLAS), bf16 in/out, fp32 accumulate"}
 
 
 def time_steps(step, steps, world, stream, sampler=None):
@@ -551,6 +599,10 @@ def main():
                          "(default), or also W in and the gradients out")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cublas-floor", action="store_true",
+                    help="also time the shape's three bare GEMMs in cuBLAS, alternating with "
+                         "the fused call (adds \"cublas_3gemm\" to the line)")
+    ap.add_argument("--floor-rounds", type=int, default=4)
     ap.add_argument("--ragged-reps", type=int, default=3)
     ap.add_argument("--ragged-limit", type=int, default=0)
     ap.add_argument("--prof-steps", type=int, default=20,
@@ -793,6 +845,8 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_sample(w, X, W, labels, args.cpu_rows)
+    floor = (cublas_floor(w, X, W, compute, stream, args.floor_rounds)
+             if args.cublas_floor and world == 1 and w.dtype == "bf16" and not dp_mode else None)
 
     if rank == 0:
         line = {"metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
@@ -813,6 +867,8 @@ def main():
                 "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps,
                 "clocks": clocks}
+        if floor is not None:
+            line["cublas_3gemm"] = floor
         print(json.dumps(line), flush=True)
     finish(world)
 

@@ -519,6 +519,7 @@ struct GemmArgs {
   int a_mn_off = 0, a_k_off = 0, b_mn_off = 0, b_k_off = 0;
   int k_splits = 1;  // CTA-pair kernels only (EPI_DX slabs)
   bool wide_epi = false;  // CTA pairs: eight epilogue warps for the exponential epilogues
+  int k_serp = 0;         // CTA pairs: alternate the K direction every k_serp tiles
 };
 
 // `c` is the TMA map of the bf16 output the CTA-pair epilogue stores (q, G,
@@ -540,6 +541,7 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
   sh.b_mn_off = g.b_mn_off;
   sh.b_k_off = g.b_k_off;
   sh.k_splits = pair ? g.k_splits : 1;
+  sh.k_serp = pair ? g.k_serp : 0;
   if (pair) {
     // Eight epilogue warps for the split-K dX slabs, and for the exponential
     // epilogues when the caller asks (short K: the epilogue, not the MMA,
@@ -832,6 +834,15 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
   return FLCE_OK;
 }
 
+// K order of a dW GEMM (M = V, N = H, K = rows).  Each wave of the
+// kPlanPairs concurrent pair tiles covers a few vocabulary tiles against all
+// of Xs (K x H).  When Xs is larger than the 46 MiB that stay in L2 beside
+// the streaming P, consecutive waves walk K in opposite directions, so a
+// wave starts on the rows of Xs the previous one ended with.
+int dw_k_serp(int64_t K, int64_t H) {
+  return K * H * 2 > (int64_t(46) << 20) ? kPlanPairs : 0;
+}
+
 // flce_fused, fused-in-forward schedule (6*BT*H*V FLOP: no logit recompute).
 // For each chunk of Cb rows:
 //   lse_q GEMM   X_b W^T; epilogue stores q = exp(y - R) dy/dz (bf16) into P
@@ -846,8 +857,10 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
 //                nothing is flagged)
 //   lse_q pass 2 the flagged rows as in pass 1
 //   dX GEMM      dX_b = f (dloss / N) (P W)   (K = all of V; bf16 out)
-//   dW GEMM      dW  (+)= (dloss / N) P^T Xs  (fp32 running sum over chunks,
-//                bf16 -- or the fp32 sum -- on the last chunk)
+// and after every dw_group chunks (P and Xs hold that many)
+//   dW GEMM      dW (+)= (dloss / N) P^T Xs over those chunks' rows: one GEMM
+//                over every row, or one per chunk into an fp32 running sum
+//                (bf16 -- or the fp32 sum -- after the last chunk)
 // then the loss over all rows.  P is never rewritten in full: the only pass
 // over it besides the two GEMMs that read it is one bf16 store per row.
 // Labels were checked by the caller.
@@ -997,6 +1010,7 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
           if (!ok) return FLCE_ERR_CUDA;
           GemmArgs gs{vn, H, grows, false};
           gs.a_mn_off = int(v0);
+          gs.k_serp = dw_k_serp(grows, H);
           FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, mo, gs, es, sms, st,
                                                     K_DWACC_GEMM)));
         }
@@ -1004,6 +1018,7 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
       }
     } else {
       GemmArgs gw{V, H, grows, false};
+      gw.k_serp = dw_k_serp(grows, H);
       FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, ew.dx_last ? mdw_out : macc, gw,
                                                 ew, sms, st, K_DWACC_GEMM)));
     }

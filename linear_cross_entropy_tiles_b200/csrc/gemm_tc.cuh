@@ -68,6 +68,8 @@ struct TcShape {
   int a_mn_off, a_k_off;    // added to A's M and K coordinates
   int b_mn_off, b_k_off;    // added to B's N and K coordinates
   int k_splits;             // > 1: K is split; split s writes fp32 slab s (EPI_DX only)
+  int k_serp;               // > 0: tile t (counted over the whole M, a_mn_off included)
+                            // walks K backwards when (t / k_serp) is odd
 };
 
 struct TcEpi {

@@ -400,7 +400,10 @@ def test_dw_once_three_chunks_matches_per_chunk(cuda_device):
     """Three row chunks (1024, 1024 and a ragged 852 rows: H = 16384 keeps a
     chunk's X rows within 46 MiB): one dW GEMM over all 2900 rows against
     three summed in fp32, with the fp32 dW too; loss and dX bitwise equal,
-    dW equal up to the order of the fp32 sums."""
+    dW equal up to the order of the fp32 sums.  The one dW GEMM's Xs (95 MB)
+    exceeds what stays in L2, so its waves of tiles alternate their K
+    direction; a tile's direction follows its place in the whole dW, so the
+    same GEMM in vocabulary slices gives the same bits."""
     BT, H, V = 2900, 16384, 500
     X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.02, 0.05, 43, device=cuda_device)
     res = {}
@@ -422,3 +425,9 @@ def test_dw_once_three_chunks_matches_per_chunk(cuda_device):
         assert float((da - db).norm() / db.norm()) <= (2e-3 if not dw32 else 1e-5)
     # the bf16 dW is the rounding of the fp32 one
     assert torch.equal(res["once", True][2].to(torch.bfloat16), res["once", False][2])
+    events = [torch.cuda.Event() for _ in range(2)]
+    with schedule(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE):
+        sliced = flce.fused(X, W, lab, softcap=5.0, dloss=0.5, slice_events=events)
+    torch.cuda.synchronize()
+    for a, b in zip(sliced, res["once", False]):
+        assert torch.equal(a, b)
