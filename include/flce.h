@@ -110,9 +110,10 @@ typedef struct {
   int32_t dw_fp32;      /* 0: dW has X's element type; 1: dW is fp32 (V x H
                            float, row stride lddw) whatever X's type, for a
                            gradient kept, or summed over ranks, in fp32.  With
-                           bf16 inputs the fused-in-forward schedule then keeps
-                           its running sum of dW in dW itself instead of the
-                           workspace.  Other values: FLCE_ERR_INVALID_ARG */
+                           bf16 inputs and one dW GEMM per row chunk the
+                           fused-in-forward schedule then keeps its running
+                           sum of dW in dW itself instead of the workspace.
+                           Other values: FLCE_ERR_INVALID_ARG */
   int64_t ldx;          /* row stride of X in elements; 0 = H */
   int64_t ldw;          /* row stride of W in elements; 0 = H */
   int64_t lddx;         /* row stride of dX in elements; 0 = H */
