@@ -2,7 +2,12 @@
 // fused linear cross-entropy library.  The operation and every entry point
 // are documented in include/flce.h.
 //
-// Schedule (two passes over the vocabulary, nothing of size BT x V in HBM):
+// Two schedules.  flce_fused on bf16 problems of 512 rows or more runs the
+// fused-in-forward schedule (6*BT*H*V FLOP), described above
+// enqueue_fused_forward: row chunks whose forward GEMM keeps q = exp(y), then
+// dX per chunk and dW over every row or per chunk.  The forward and backward
+// entry points, fp32 problems and small batches run the recompute schedule
+// (two passes over the vocabulary, nothing of size BT x V in HBM):
 //   forward   labels_kernel -> logit GEMM X W^T with the online-LSE epilogue
 //             (per-(tile,row) max / sum-exp partials + target logit)
 //             -> combine_kernel (lse, per-row NLL) -> finalize_kernel (loss)

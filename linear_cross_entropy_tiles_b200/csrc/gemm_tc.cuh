@@ -54,7 +54,8 @@ constexpr int kStatusTimeout = 6;  // FLCE_ERR_TIMEOUT
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 // EPI_DX is the generic "fp32 running sum across launches" epilogue: it also
-// accumulates dW over row chunks in the fused-in-forward schedule.
+// accumulates dW over row chunks in the fused-in-forward schedule, or writes
+// it in a single pass when one GEMM covers every row.
 // The *_CAP modes are the same epilogues with the logit softcap compiled in.
 enum : int {
   EPI_LSE = 0, EPI_GRAD = 1, EPI_DX = 2, EPI_DW = 3, EPI_LSE_Q = 4,

@@ -307,6 +307,40 @@ def test_workspace_below_one_logits_tensor_when_capped_or_fp32_dW(name):
         assert free == f32 and q_all < free < per_chunk and free < 1.2 * logits_bytes
 
 
+@pytest.mark.parametrize("name,once", [("llama3_8b", True), ("gemma2_softcap", True),
+                                       ("gpt2_small", False)])
+def test_dw_passes_chosen_by_the_memory_rule_on_the_bench_shapes(name, once):
+    """The automatic plan's dW passes on the benchmark shapes: one dW GEMM
+    over every row where all rows' q takes no more than one chunk's q plus
+    the fp32 V x H sum (Llama-3: 2.10 <= 1.05 + 2.10 GB; Gemma2: 4.19 <=
+    2.10 + 3.67 GB), one per chunk where it would take more (GPT-2: 3.30 >
+    0.83 + 0.15 GB); on the ragged sweep the rule picks one dW GEMM up to
+    about 12k rows."""
+    w = inputs.WORKLOADS[name]
+    p = flce.make_problem(w.BT, w.H, w.V, flce.FLCE_BF16, softcap=w.softcap)
+
+    def size(schedule, prob=p):
+        old = flce.flce_set_schedule(schedule)
+        try:
+            return flce.flce_workspace_size(prob, flce.FLCE_OP_FUSED)
+        finally:
+            flce.flce_set_schedule(old)
+
+    auto = size(flce.FLCE_SCHEDULE_AUTO)
+    assert auto == size(flce.FLCE_SCHEDULE_FUSED_FORWARD)
+    assert auto == size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE if once
+                        else flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK)
+    if name == "llama3_8b":
+        picks = []
+        for bt in inputs.ragged_bt_list():
+            q = flce.make_problem(bt, w.H, w.V, flce.FLCE_BF16)
+            picks.append((bt, size(flce.FLCE_SCHEDULE_AUTO, q) ==
+                          size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE, q)))
+        assert sum(o for _, o in picks) == 17
+        assert max(bt for bt, o in picks if o) < min(bt for bt, o in picks if not o)
+        assert 12000 < min(bt for bt, o in picks if not o) < 13000
+
+
 def test_workspace_cap_falls_back_to_per_chunk_dW_then_recompute():
     """Under a workspace cap the automatic schedule keeps the fused-in-forward
     schedule with one dW GEMM per row chunk when holding every row's q for
