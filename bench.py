@@ -54,17 +54,17 @@ METRIC = ("FLCE fwd+bwd tokens/s and TFLOP/s (% of B200 BF16 peak); peak extra H
 # are reported as null for any other build or workload.
 TRAFFIC = {
     ("llama3_8b", "auto"): {
-        "csrc_sha16": "fbcd890a5973ffee",
-        "bytes_per_launch": {"lse_q_gemm": 2.3438e9, "dx_gemm": 5.6258e9, "dw_acc_gemm": 8.4876e9,
+        "csrc_sha16": "8dea23cbe5ebac1f",
+        "bytes_per_launch": {"lse_q_gemm": 2.3815e9, "dx_gemm": 5.5945e9, "dw_acc_gemm": 5.0345e9,
                              "lse_q": 0.0255e9}},
     ("gpt2_small", "auto"): {
-        "csrc_sha16": "fbcd890a5973ffee",
-        "bytes_per_launch": {"lse_q_gemm": 0.888e9, "dx_gemm": 1.055e9,
-                             "dw_acc_gemm": 1.182e9}},
+        "csrc_sha16": "8dea23cbe5ebac1f",
+        "bytes_per_launch": {"lse_q_gemm": 0.890e9, "dx_gemm": 1.0545e9,
+                             "dw_acc_gemm": 1.183e9}},
     ("ce_llmc", "auto"): {
-        "csrc_sha16": "fbcd890a5973ffee",
-        "bytes_per_launch": {"ce_forward": 3.299e9, "ce_backward": 6.5415e9,
-                             "ce_fused": 6.530e9}},
+        "csrc_sha16": "8dea23cbe5ebac1f",
+        "bytes_per_launch": {"ce_forward": 3.298e9, "ce_backward": 6.542e9,
+                             "ce_fused": 6.531e9}},
 }
 
 
@@ -361,10 +361,6 @@ def workload_config(w, world, parallel="replicas"):
 
 
 SCHEDULE = ["auto"]
-# --schedule names: flce_set_schedule values (the fused-in-forward schedule
-# with dW passes by the library's rule, one per row chunk, or one over all rows)
-SCHEDULES = {"auto": 0, "recompute": 1, "fused_fwd": 2, "fused_fwd_dw_per_chunk": 3,
-             "fused_fwd_dw_once": 4}
 
 
 def run_ragged(args, world, rank):
@@ -374,7 +370,7 @@ def run_ragged(args, world, rank):
     import linear_cross_entropy_tiles_b200 as flce
     from linear_cross_entropy_tiles_b200 import build, inputs
     build.build()
-    flce.flce_set_schedule(SCHEDULES[args.schedule])
+    flce.flce_set_schedule({"auto": 0, "recompute": 1, "fused_fwd": 2}[args.schedule])
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream()
     bts = inputs.ragged_bt_list()
@@ -585,7 +581,7 @@ def main():
                     help="override V of an LM-head workload (small cases for profiling "
                          "that keep the full-size K of every GEMM)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--schedule", default="auto", choices=list(SCHEDULES),
+    ap.add_argument("--schedule", default="auto", choices=["auto", "recompute", "fused_fwd"],
                     help="flce_fused schedule (auto: fused-in-forward for BT >= 512)")
     ap.add_argument("--cpu-rows", type=int, default=8)
     ap.add_argument("--ce-cpu-rows", type=int, default=8192)
@@ -661,7 +657,7 @@ def main():
     if args.parallel == "dp" and world > 1:
         W = inputs.make_workload(dataclasses.replace(w, seed=inputs.WORKLOADS[args.workload].seed),
                                  device=dev, BT=1)[1]  # the same W on every rank
-    flce.flce_set_schedule(SCHEDULES[args.schedule])
+    flce.flce_set_schedule({"auto": 0, "recompute": 1, "fused_fwd": 2}[args.schedule])
     dp_mode = args.parallel == "dp"
     # Data parallel: each rank writes its dW share in fp32 and the ranks sum
     # it in fp32 (--dw-reduce bf16: bf16 shares summed in bf16).

@@ -110,10 +110,9 @@ typedef struct {
   int32_t dw_fp32;      /* 0: dW has X's element type; 1: dW is fp32 (V x H
                            float, row stride lddw) whatever X's type, for a
                            gradient kept, or summed over ranks, in fp32.  With
-                           bf16 inputs and one dW GEMM per row chunk the
-                           fused-in-forward schedule then keeps its running
-                           sum of dW in dW itself instead of the workspace.
-                           Other values: FLCE_ERR_INVALID_ARG */
+                           bf16 inputs the fused-in-forward schedule then keeps
+                           its running sum of dW in dW itself instead of the
+                           workspace.  Other values: FLCE_ERR_INVALID_ARG */
   int64_t ldx;          /* row stride of X in elements; 0 = H */
   int64_t ldw;          /* row stride of W in elements; 0 = H */
   int64_t lddx;         /* row stride of dX in elements; 0 = H */
@@ -355,21 +354,15 @@ FLCE_API flce_status_t flce_ce_fused(const flce_ce_problem_t* p, const void* log
  *  FLCE_SCHEDULE_FUSED_FORWARD: per row chunk (at least two; at most
  *    1 GiB of q, 2 GiB when an fp32 V x H array exceeds 1 GiB, and 46 MiB
  *    of X rows each) the forward GEMM keeps q = exp(y) dy/dz in bf16 against
- *    one exponent reference per row, the chunk's lse and row factors follow,
- *    and dX for the chunk is q W scaled per row (6*BT*H*V FLOP).  dW is
- *    one GEMM over every row when the q of all rows is no larger than one
- *    chunk's q plus an fp32 V x H array (workspace: that q, about one bf16
- *    BT x V tensor), else one GEMM per chunk summed in an fp32 V x H array
- *    (workspace: a chunk's q plus that array, unless dW is fp32).
- *  FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK, FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE:
- *    the same with dW always per chunk, or always over every row.
+ *    one exponent reference per row; the chunk's lse and row factors follow;
+ *    dX for the chunk is q W scaled per row, and the chunk's dW is added
+ *    into an fp32 V x H running sum (6*BT*H*V FLOP; workspace: a chunk's q
+ *    plus that sum, or only the q when dW is fp32).
  *  FLCE_SCHEDULE_AUTO: fused-in-forward when BT >= 512, else recompute. */
 typedef enum {
   FLCE_SCHEDULE_AUTO = 0,
   FLCE_SCHEDULE_RECOMPUTE = 1,
-  FLCE_SCHEDULE_FUSED_FORWARD = 2,
-  FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK = 3,
-  FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE = 4
+  FLCE_SCHEDULE_FUSED_FORWARD = 2
 } flce_schedule_t;
 
 /* Set the process-wide flce_fused schedule (also used by
@@ -380,8 +373,7 @@ FLCE_API int32_t flce_set_schedule(int32_t schedule);
 /* Process-wide cap, in bytes, on the workspace flce_fused plans under
  * FLCE_SCHEDULE_AUTO (0 = none, the default; also used by
  * flce_workspace_size for FLCE_OP_FUSED).  Under the cap AUTO takes the
- * fused-in-forward schedule only when its workspace fits (first with its
- * own choice of dW passes, then with one dW GEMM per chunk), else the
+ * fused-in-forward schedule only when its workspace fits, else the
  * recompute schedule with its vocabulary chunk narrowed (down to 256
  * columns) until the workspace fits; when nothing fits it plans the
  * smallest recompute workspace.  A cap of one bf16 BT x V tensor (2*BT*V

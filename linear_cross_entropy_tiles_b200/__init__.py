@@ -10,7 +10,6 @@ from .binding import (ce_backward, ce_forward, ce_fused, ce_workspace, flce_ce_b
                       flce_ce_forward, flce_ce_problem_t, flce_ce_workspace_size,
                       make_ce_problem)
 from .binding import (FLCE_BF16, FLCE_FP32, FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_FUSED_FORWARD,
-                      FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE, FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK,
                       FLCE_SCHEDULE_RECOMPUTE, FLCE_OP_BACKWARD, FLCE_OP_FORWARD, FLCE_OP_FUSED,
                       FlceError, backward, count_valid, flce_backward, flce_count_valid,
                       dw_slice_bounds, flce_dw_slice_rows, flce_forward, flce_fused,

@@ -40,7 +40,6 @@ EXPORTS = ("flce_workspace_size", "flce_forward", "flce_backward", "flce_fused",
            "flce_vp_workspace_size", "flce_vp_forward", "flce_vp_combine", "flce_vp_backward",
            "flce_fused_global_sliced", "flce_dw_slice_rows")
 FLCE_SCHEDULE_AUTO, FLCE_SCHEDULE_RECOMPUTE, FLCE_SCHEDULE_FUSED_FORWARD = 0, 1, 2
-FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK, FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE = 3, 4
 
 
 class FlceError(RuntimeError):

@@ -5,9 +5,9 @@
 // Two schedules.  flce_fused on bf16 problems of 512 rows or more runs the
 // fused-in-forward schedule (6*BT*H*V FLOP), described above
 // enqueue_fused_forward: row chunks whose forward GEMM keeps q = exp(y), then
-// dX per chunk and dW over every row or per chunk.  The forward and backward
-// entry points, fp32 problems and small batches run the recompute schedule
-// (two passes over the vocabulary, nothing of size BT x V in HBM):
+// dX and dW per chunk.  The forward and backward entry points, fp32 problems
+// and small batches run the recompute schedule (two passes over the
+// vocabulary, nothing of size BT x V in HBM):
 //   forward   labels_kernel -> logit GEMM X W^T with the online-LSE epilogue
 //             (per-(tile,row) max / sum-exp partials + target logit)
 //             -> combine_kernel (lse, per-row NLL) -> finalize_kernel (loss)
@@ -116,11 +116,9 @@ struct Plan {
   size_t off_lse = 0, off_target = 0, off_rowloss = 0, off_partial = 0, off_g = 0,
          off_dxacc = 0, total = 0;
   // fused-in-forward schedule (flce_fused, bf16): row chunks of Cb rows whose
-  // p = exp(y - reference) live in P [dw_group * Cb][ldp]; one dW GEMM per
-  // dw_group chunks over their rows, summed in fp32 when there are several
+  // p = exp(y - reference) live in P [Cb][ldp]; dW summed in fp32 over chunks
   bool fused_fwd = false;
   int64_t Cb = 0, n_row_chunks = 0, ldp = 0;
-  int64_t dw_group = 1;   // row chunks whose q and Xs are held for one dW GEMM
   int dx_splits = 1;      // K (vocabulary) splits of the chunk's dX GEMM
   size_t off_p = 0, off_dwacc = 0, off_dxslab = 0;
   // per chunk row: prescaled X rows [Cb][H] bf16, exponent reference and dX
@@ -205,16 +203,12 @@ int pick_k_splits(int64_t tiles, int pairs, int64_t k_stages) {
 bool use_fused_forward(const flce_problem_t* p) {
   if (p->dtype != FLCE_BF16 || p->BT <= 0) return false;
   const int32_t s = g_schedule.load();
-  if (s == FLCE_SCHEDULE_RECOMPUTE) return false;
-  if (s != FLCE_SCHEDULE_AUTO) return true;  // the fused-in-forward schedules
+  if (s == 1) return false;
+  if (s == 2) return true;
   return p->BT >= 512;
 }
 
-// dW passes of the fused-in-forward schedule: chosen by the rule below, one
-// per row chunk (an fp32 running sum), or one over every row.
-enum DwPasses { kDwAuto = 0, kDwPerChunk = 1, kDwOnce = 2 };
-
-void make_plan_fused_forward(const flce_problem_t* p, Plan* pl, int dw_passes) {
+void make_plan_fused_forward(const flce_problem_t* p, Plan* pl) {
   const int64_t BT = p->BT, V = p->V, H = p->H;
   pl->BT = BT;
   pl->H = H;
@@ -243,19 +237,6 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl, int dw_passes) {
   if (x_rows >= 128 && cdiv(BT, x_rows) > n) n = cdiv(BT, x_rows);
   pl->Cb = round_up(cdiv(BT, n), 128);
   pl->n_row_chunks = cdiv(BT, pl->Cb);
-  // One dW GEMM over every row (K = BT) instead of one per chunk when the q
-  // of all rows takes no more memory than a chunk's q plus the V x H fp32
-  // sum the per-chunk passes accumulate in: that sum's read-modify-write
-  // (4.2 GB per chunk on the Llama-3 shape) is gone and dW is written once.
-  // The forward and dX GEMMs keep their chunks (X rows blocked in L2).
-  const int64_t nch = pl->n_row_chunks;
-  const size_t q_all = size_t(BT) * size_t(pl->ldp) * 2;
-  const size_t q_chunk = size_t(pl->Cb) * size_t(pl->ldp) * 2;
-  const bool once = nch > 1 && (dw_passes == kDwOnce ||
-                                (dw_passes == kDwAuto &&
-                                 q_all <= q_chunk + size_t(V) * size_t(H) * 4));
-  pl->dw_group = once ? nch : 1;
-  const size_t held = size_t(pl->dw_group) * size_t(pl->Cb);  // rows of q and Xs
   size_t off = kHeaderBytes;
   const size_t rows = size_t(BT);
   pl->off_lse = off;
@@ -267,9 +248,9 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl, int dw_passes) {
   pl->off_partial = off;
   off = align256(off + size_t(pl->part_tiles) * rows * 8);
   pl->off_p = off;
-  off = align256(off + held * size_t(pl->ldp) * 2);
-  // The fp32 running sum of dW over the dW passes, unless dW itself is fp32.
-  if (cdiv(nch, pl->dw_group) > 1 && !p->dw_fp32) {
+  off = align256(off + size_t(pl->Cb) * size_t(pl->ldp) * 2);
+  // The fp32 running sum of dW over row chunks, unless dW itself is fp32.
+  if (pl->n_row_chunks > 1 && !p->dw_fp32) {
     pl->off_dwacc = off;
     off = align256(off + size_t(V) * size_t(H) * 4);
   }
@@ -282,7 +263,7 @@ void make_plan_fused_forward(const flce_problem_t* p, Plan* pl, int dw_passes) {
   }
   const size_t cb = size_t(pl->Cb);
   pl->off_xs = off;
-  off = align256(off + held * size_t(H) * 2);
+  off = align256(off + cb * size_t(H) * 2);
   pl->off_ref = off;
   off = align256(off + cb * 4);
   pl->off_rowscale = off;
@@ -305,10 +286,6 @@ void make_plan(const flce_problem_t* p, int op, Plan* pl) {
   const size_t extra = p->shift_seq_len > 0 ? align256(size_t(p->BT) * 8) : 0;
   const unsigned long long limit = g_schedule.load() == 0 ? g_ws_limit.load() : 0ull;
   make_plan_base(p, op, pl, 32768);
-  if (limit && pl->fused_fwd && pl->dw_group > 1 && pl->total + extra > limit) {
-    *pl = Plan{};
-    make_plan_fused_forward(p, pl, kDwPerChunk);  // q of one chunk at a time
-  }
   if (limit && op == FLCE_OP_FUSED && p->dtype == FLCE_BF16 && pl->total + extra > limit) {
     for (int64_t vc = 32768; vc >= 256; vc /= 2) {
       *pl = Plan{};
@@ -332,11 +309,7 @@ void make_plan(const flce_problem_t* p, int op, Plan* pl) {
 // sum (no workspace for it).
 void make_plan_base(const flce_problem_t* p, int op, Plan* pl, int64_t vc_max) {
   if (op == FLCE_OP_FUSED && use_fused_forward(p)) {
-    const int32_t s = g_schedule.load();
-    make_plan_fused_forward(p, pl,
-                            s == FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK ? kDwPerChunk
-                            : s == FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE    ? kDwOnce
-                                                                          : kDwAuto);
+    make_plan_fused_forward(p, pl);
     return;
   }
   if (op == FLCE_OP_FUSED + 16) op = FLCE_OP_FUSED;
@@ -524,7 +497,6 @@ struct GemmArgs {
   int a_mn_off = 0, a_k_off = 0, b_mn_off = 0, b_k_off = 0;
   int k_splits = 1;  // CTA-pair kernels only (EPI_DX slabs)
   bool wide_epi = false;  // CTA pairs: eight epilogue warps for the exponential epilogues
-  int k_serp = 0;         // CTA pairs: alternate the K direction every k_serp tiles
 };
 
 // `c` is the TMA map of the bf16 output the CTA-pair epilogue stores (q, G,
@@ -546,7 +518,6 @@ cudaError_t launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtens
   sh.b_mn_off = g.b_mn_off;
   sh.b_k_off = g.b_k_off;
   sh.k_splits = pair ? g.k_splits : 1;
-  sh.k_serp = pair ? g.k_serp : 0;
   if (pair) {
     // Eight epilogue warps for the split-K dX slabs, and for the exponential
     // epilogues when the caller asks (short K: the epilogue, not the MMA,
@@ -839,15 +810,6 @@ flce_status_t enqueue_backward(const flce_problem_t* p, const Plan& pl, const Pt
   return FLCE_OK;
 }
 
-// K order of a dW GEMM (M = V, N = H, K = rows).  Each wave of the
-// kPlanPairs concurrent pair tiles covers a few vocabulary tiles against all
-// of Xs (K x H).  When Xs is larger than the 46 MiB that stay in L2 beside
-// the streaming P, consecutive waves walk K in opposite directions, so a
-// wave starts on the rows of Xs the previous one ended with.
-int dw_k_serp(int64_t K, int64_t H) {
-  return K * H * 2 > (int64_t(46) << 20) ? kPlanPairs : 0;
-}
-
 // flce_fused, fused-in-forward schedule (6*BT*H*V FLOP: no logit recompute).
 // For each chunk of Cb rows:
 //   lse_q GEMM   X_b W^T; epilogue stores q = exp(y - R) dy/dz (bf16) into P
@@ -862,10 +824,8 @@ int dw_k_serp(int64_t K, int64_t H) {
 //                nothing is flagged)
 //   lse_q pass 2 the flagged rows as in pass 1
 //   dX GEMM      dX_b = f (dloss / N) (P W)   (K = all of V; bf16 out)
-// and after every dw_group chunks (P and Xs hold that many)
-//   dW GEMM      dW (+)= (dloss / N) P^T Xs over those chunks' rows: one GEMM
-//                over every row, or one per chunk into an fp32 running sum
-//                (bf16 -- or the fp32 sum -- after the last chunk)
+//   dW GEMM      dW  (+)= (dloss / N) P^T Xs  (fp32 running sum over chunks,
+//                bf16 -- or the fp32 sum -- on the last chunk)
 // then the loss over all rows.  P is never rewritten in full: the only pass
 // over it besides the two GEMMs that read it is one bf16 store per row.
 // Labels were checked by the caller.
@@ -897,13 +857,11 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
   for (int64_t b = 0; b < pl.n_row_chunks; ++b) {
     const int64_t row0 = b * pl.Cb;
     const int64_t rows = (BT - row0) < pl.Cb ? (BT - row0) : pl.Cb;
-    // The chunk's q and Xs rows: slot b mod dw_group of the held rows.
-    const int64_t slot = b % pl.dw_group;
-    __nv_bfloat16* Pb = P + slot * pl.Cb * pl.ldp;
-    __nv_bfloat16* Xsb = Xs + slot * pl.Cb * H;
-    CUtensorMap mp_k, mp_out, mdx_out;
-    if (!(make_map(&mp_k, Pb, pl.ldp, rows, pl.ldp * 2, 64, kBM) &&
-          make_map(&mp_out, Pb, pl.ldp, rows, pl.ldp * 2, 64, 32) &&
+    CUtensorMap mp_k, mp_mn, mp_out, mdx_out, mxs_mn;
+    if (!(make_map(&mp_k, P, pl.ldp, rows, pl.ldp * 2, 64, kBM) &&
+          make_map(&mp_mn, P, pl.ldp, rows, pl.ldp * 2, 64, 64) &&
+          make_map(&mp_out, P, pl.ldp, rows, pl.ldp * 2, 64, 32) &&
+          make_map(&mxs_mn, Xs, H, rows, H * 2, 64, 64) &&
           make_map(&mdx_out, static_cast<__nv_bfloat16*>(q.dX) + row0 * pl.lddx, H, rows,
                    pl.lddx * 2, 64, 32)))
       return FLCE_ERR_CUDA;
@@ -911,7 +869,7 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     ep.partial = partial;
     ep.target = target;
     ep.row0 = row0;
-    ep.P = Pb;
+    ep.P = P;
     ep.ldp = pl.ldp;
     ep.out_cols = int(pl.ldp);
     GemmArgs gf{rows, V, H, true};
@@ -934,8 +892,8 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
                                                        kind)));
       prof_before(st);
       lse_q_kernel<<<groups, kLseQThreads, 0, st>>>(
-          pass, partial, int(pl.part_tiles), BT, row0, rows, target, q.labels, p->ignore_index, Pb,
-          pl.ldp, static_cast<const __nv_bfloat16*>(q.X), pl.ldx, H, Xsb, ref, flags, lse,
+          pass, partial, int(pl.part_tiles), BT, row0, rows, target, q.labels, p->ignore_index, P,
+          pl.ldp, static_cast<const __nv_bfloat16*>(q.X), pl.ldx, H, Xs, ref, flags, lse,
           rowloss, row_scale, hdr, q.dloss_host, cap);
       prof_after(st, K_LSEQ);
       FLCE_TRY(cudaGetLastError());
@@ -963,16 +921,8 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
       prof_after(st, K_DX_REDUCE);
       FLCE_TRY(cudaGetLastError());
     }
-    // dW += (dloss / N) P^T Xs over the rows of the held chunks, once the
-    // last of them is done: one GEMM over every row, or one per chunk into
-    // an fp32 running sum (in the workspace, or in dW itself when dW is fp32)
-    if (slot != pl.dw_group - 1 && b != pl.n_row_chunks - 1) continue;
-    const int64_t grow0 = (b - slot) * pl.Cb;  // the group's first row
-    const int64_t grows = row0 + rows - grow0;  // its rows: K of the dW GEMM
-    CUtensorMap mp_mn, mxs_mn;
-    if (!(make_map(&mp_mn, P, pl.ldp, grows, pl.ldp * 2, 64, 64) &&
-          make_map(&mxs_mn, Xs, H, grows, H * 2, 64, 64)))
-      return FLCE_ERR_CUDA;
+    // dW += (dloss / N) P^T Xs: an fp32 running sum over the row chunks, in
+    // the workspace, or in dW itself when dW is fp32
     TcEpi ew = ep;
     ew.dx_acc = pl.dw_f32 ? static_cast<float*>(q.dW)
                           : reinterpret_cast<float*>(q.ws + pl.off_dwacc);
@@ -980,7 +930,7 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
     ew.out_f32 = pl.dw_f32 ? 1 : 0;
     ew.dx = static_cast<__nv_bfloat16*>(q.dW);
     ew.ld_dx = pl.lddw;
-    ew.dx_first = grow0 == 0;
+    ew.dx_first = b == 0;
     ew.dx_last = b == pl.n_row_chunks - 1;
     ew.out_cols = int(H);
     ew.scale_by_nvalid = 1;
@@ -1013,17 +963,15 @@ flce_status_t enqueue_fused_forward(const flce_problem_t* p, const Plan& pl, con
                               : make_map(&mo, static_cast<__nv_bfloat16*>(q.dW) + v0 * pl.lddw,
                                          H, vn, pl.lddw * 2, 64, 32);
           if (!ok) return FLCE_ERR_CUDA;
-          GemmArgs gs{vn, H, grows, false};
+          GemmArgs gs{vn, H, rows, false};
           gs.a_mn_off = int(v0);
-          gs.k_serp = dw_k_serp(grows, H);
           FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, mo, gs, es, sms, st,
                                                     K_DWACC_GEMM)));
         }
         if (cudaEventRecord(q.slice_done[sl], st) != cudaSuccess) return FLCE_ERR_CUDA;
       }
     } else {
-      GemmArgs gw{V, H, grows, false};
-      gw.k_serp = dw_k_serp(grows, H);
+      GemmArgs gw{V, H, rows, false};
       FLCE_TRY((launch_gemm<true, true, EPI_DX>(mp_mn, mxs_mn, ew.dx_last ? mdw_out : macc, gw,
                                                 ew, sms, st, K_DWACC_GEMM)));
     }
@@ -1288,7 +1236,7 @@ flce_status_t flce_selftest_approx(const float* x, int64_t n, float* out, struct
 uint64_t flce_set_workspace_limit(uint64_t bytes) { return g_ws_limit.exchange(bytes); }
 
 int32_t flce_set_schedule(int32_t schedule) {
-  if (schedule < FLCE_SCHEDULE_AUTO || schedule > FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE) return -1;
+  if (schedule < FLCE_SCHEDULE_AUTO || schedule > FLCE_SCHEDULE_FUSED_FORWARD) return -1;
   return g_schedule.exchange(schedule);
 }
 

@@ -13,8 +13,7 @@
 // call left in it.  The fused computation writes every scratch byte it later
 // reads within the same call (the status word, N_valid, the shifted labels,
 // the LSE partials, the q / G chunk, the dX accumulator or split slabs, and
-// the dW running sum where the plan has one, whose first pass stores
-// without reading), so
+// the dW running sum, whose first row chunk stores without reading), so
 // nothing has to be cleared between calls.  Two calls whose GPU work overlaps in time (different streams, or
 // different host threads on the same device) race on the array and give
 // wrong results; serialise them.

@@ -54,8 +54,7 @@ constexpr int kStatusTimeout = 6;  // FLCE_ERR_TIMEOUT
 constexpr uint64_t kDrainLimitNs = 1000000000ull;
 
 // EPI_DX is the generic "fp32 running sum across launches" epilogue: it also
-// accumulates dW over row chunks in the fused-in-forward schedule, or writes
-// it in a single pass when one GEMM covers every row.
+// accumulates dW over row chunks in the fused-in-forward schedule.
 // The *_CAP modes are the same epilogues with the logit softcap compiled in.
 enum : int {
   EPI_LSE = 0, EPI_GRAD = 1, EPI_DX = 2, EPI_DW = 3, EPI_LSE_Q = 4,
@@ -69,8 +68,6 @@ struct TcShape {
   int a_mn_off, a_k_off;    // added to A's M and K coordinates
   int b_mn_off, b_k_off;    // added to B's N and K coordinates
   int k_splits;             // > 1: K is split; split s writes fp32 slab s (EPI_DX only)
-  int k_serp;               // > 0: tile t (counted over the whole M, a_mn_off included)
-                            // walks K backwards when (t / k_serp) is odd
 };
 
 struct TcEpi {

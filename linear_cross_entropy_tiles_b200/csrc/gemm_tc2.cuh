@@ -137,14 +137,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(tc2_threads(EW), 1)
       if (!tile_wanted(ep, sh, mt * kPairBM, kPairBM)) continue;
       const int m0 = mt * kPairBM + 128 * int(rank) + sh.a_mn_off;
       const int n0 = nt * kPairBN + 128 * int(rank) + sh.b_mn_off;
-      const int kb0 = split * kps;
-      const int kb1 = min(k_stages, kb0 + kps);
-      // The K order of this tile (the MMA issuer only counts stages, so the
-      // sum is the same set of products in the order loaded here).
-      const bool rev = sh.k_serp > 0 &&
-                       ((((mt + sh.a_mn_off / kPairBM) * sh.n_tiles + nt) / sh.k_serp) & 1);
-      for (int kq = kb0; kq < kb1; ++kq) {
-        const int kb = rev ? kb0 + kb1 - 1 - kq : kq;
+      const int kb1 = min(k_stages, (split + 1) * kps);
+      for (int kb = split * kps; kb < kb1; ++kb) {
         if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, abort_flag)) {
           record_timeout(ep, abort_flag);
           ok = false;

@@ -258,14 +258,10 @@ def test_binding_checks_tensors_against_the_problem():
 @pytest.mark.parametrize("name", ["gpt2_small", "llama3_8b", "gemma2_softcap"])
 def test_workspace_below_one_logits_tensor_when_capped_or_fp32_dW(name):
     """The survey's bound on peak extra HBM, below one bf16 BT x V tensor,
-    holds under a workspace cap of exactly that size, for a bf16 or an fp32
-    dW (the automatic schedule then takes one dW GEMM per row chunk, gives
-    up the fused-in-forward plan, or narrows the recompute chunk, as
-    needed).  Uncapped, the automatic plan holds every row's q for one dW
-    GEMM when that takes no more than a chunk's q plus the fp32 V x H sum
-    (Llama-3, Gemma2: about one logits tensor), else sums per chunk
-    (GPT-2); with one dW GEMM per chunk an fp32 dW is its own running sum,
-    so the workspace shrinks by exactly that sum."""
+    holds in two modes: under a workspace cap of exactly that size (the
+    automatic schedule then gives up the fused-in-forward plan, or narrows
+    the recompute chunk, as needed), and with an fp32 dW, where the
+    fused-in-forward schedule keeps its running sum in dW itself."""
     w = inputs.WORKLOADS[name]
     logits_bytes = 2 * w.BT * w.V
     p = flce.make_problem(w.BT, w.H, w.V, flce.FLCE_BF16, softcap=w.softcap)
@@ -286,85 +282,8 @@ def test_workspace_below_one_logits_tensor_when_capped_or_fp32_dW(name):
     assert forced == free and 0 < smallest <= capped
     p32 = flce.make_problem(w.BT, w.H, w.V, flce.FLCE_BF16, softcap=w.softcap, dw_fp32=1)
     f32 = flce.flce_workspace_size(p32, flce.FLCE_OP_FUSED)
-    prev = flce.flce_set_workspace_limit(logits_bytes)
-    try:
-        f32_capped = flce.flce_workspace_size(p32, flce.FLCE_OP_FUSED)
-    finally:
-        flce.flce_set_workspace_limit(prev)
-    old = flce.flce_set_schedule(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK)
-    try:
-        per_chunk = flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
-        per_chunk32 = flce.flce_workspace_size(p32, flce.FLCE_OP_FUSED)
-    finally:
-        flce.flce_set_schedule(old)
-    sum32 = -(-w.V * w.H * 4 // 256) * 256
-    assert f32_capped < logits_bytes
-    assert per_chunk - per_chunk32 == sum32                # exactly the fp32 sum
-    q_all = 2 * w.BT * (-(-w.V // 256) * 256)
-    if name == "gpt2_small":                               # per chunk: a small fp32 sum
-        assert free == per_chunk and f32 == per_chunk32
-    else:                                                  # one dW GEMM over every row
-        assert free == f32 and q_all < free < per_chunk and free < 1.2 * logits_bytes
-
-
-@pytest.mark.parametrize("name,once", [("llama3_8b", True), ("gemma2_softcap", True),
-                                       ("gpt2_small", False)])
-def test_dw_passes_chosen_by_the_memory_rule_on_the_bench_shapes(name, once):
-    """The automatic plan's dW passes on the benchmark shapes: one dW GEMM
-    over every row where all rows' q takes no more than one chunk's q plus
-    the fp32 V x H sum (Llama-3: 2.10 <= 1.05 + 2.10 GB; Gemma2: 4.19 <=
-    2.10 + 3.67 GB), one per chunk where it would take more (GPT-2: 3.30 >
-    0.83 + 0.15 GB); on the ragged sweep the rule picks one dW GEMM up to
-    about 12k rows."""
-    w = inputs.WORKLOADS[name]
-    p = flce.make_problem(w.BT, w.H, w.V, flce.FLCE_BF16, softcap=w.softcap)
-
-    def size(schedule, prob=p):
-        old = flce.flce_set_schedule(schedule)
-        try:
-            return flce.flce_workspace_size(prob, flce.FLCE_OP_FUSED)
-        finally:
-            flce.flce_set_schedule(old)
-
-    auto = size(flce.FLCE_SCHEDULE_AUTO)
-    assert auto == size(flce.FLCE_SCHEDULE_FUSED_FORWARD)
-    assert auto == size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE if once
-                        else flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK)
-    if name == "llama3_8b":
-        picks = []
-        for bt in inputs.ragged_bt_list():
-            q = flce.make_problem(bt, w.H, w.V, flce.FLCE_BF16)
-            picks.append((bt, size(flce.FLCE_SCHEDULE_AUTO, q) ==
-                          size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE, q)))
-        assert sum(o for _, o in picks) == 17
-        assert max(bt for bt, o in picks if o) < min(bt for bt, o in picks if not o)
-        assert 12000 < min(bt for bt, o in picks if not o) < 13000
-
-
-def test_workspace_cap_falls_back_to_per_chunk_dW_then_recompute():
-    """Under a workspace cap the automatic schedule keeps the fused-in-forward
-    schedule with one dW GEMM per row chunk when holding every row's q for
-    one dW GEMM does not fit, before it gives the schedule up (BT = 12345 on
-    the Llama-3 shape: 3.68 GB for one dW GEMM, 3.55 GB per chunk)."""
-    p = flce.make_problem(12345, 4096, 128256, flce.FLCE_BF16)
-
-    def size(schedule, cap):
-        old_s = flce.flce_set_schedule(schedule)
-        old_c = flce.flce_set_workspace_limit(cap)
-        try:
-            return flce.flce_workspace_size(p, flce.FLCE_OP_FUSED)
-        finally:
-            flce.flce_set_workspace_limit(old_c)
-            flce.flce_set_schedule(old_s)
-
-    once = size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE, 0)
-    per_chunk = size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK, 0)
-    auto = flce.FLCE_SCHEDULE_AUTO
-    assert per_chunk < once and size(auto, 0) == once == size(auto, once)
-    assert size(auto, once - 1) == per_chunk == size(auto, per_chunk)
-    assert size(auto, per_chunk - 1) < per_chunk            # the recompute plan
-    # forced schedules ignore the cap
-    assert size(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE, 1) == once
+    assert f32 < logits_bytes
+    assert free - f32 == -(-w.V * w.H * 4 // 256) * 256     # exactly the fp32 sum
 
 
 def test_dw_fp32_problem_checks():

@@ -102,22 +102,19 @@ def test_fused_dp_one_rank_nccl_equals_fused(cuda_device):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("sched", ["recompute", "fused_fwd", "fused_fwd_dw_once"])
+@pytest.mark.parametrize("sched", ["recompute", "fused_fwd"])
 @pytest.mark.parametrize("n_slices,dw_fp32", [(1, False), (4, False), (8, False), (3, True)])
 def test_sliced_dW_equals_unsliced(sched, n_slices, dw_fp32, cuda_device):
-    """flce_fused_global_sliced: the last dW GEMM in vocabulary slices of
-    whole 256-row tiles computes the same tiles in the same order, so loss,
-    dX and dW equal flce_fused's bit for bit (V = 3000 in 8 slices of 512
-    rows leaves two empty); every slice's event is recorded; the
+    """flce_fused_global_sliced: the last row chunk's dW GEMM in vocabulary
+    slices of whole 256-row tiles computes the same tiles in the same order,
+    so loss, dX and dW equal flce_fused's bit for bit (V = 3000 in 8 slices
+    of 512 rows leaves two empty); every slice's event is recorded; the
     fused-in-forward schedule launches one dW GEMM per non-empty slice in
-    its last dW pass (the last row chunk's, or the one over every row), and
-    dW may be a row-strided view."""
+    its last row chunk, and dW may be a row-strided view."""
     BT, H, V, cap = 1100, 128, 3000, 5.0
     X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.05, 0.1, 65, device=cuda_device)
     prev = flce.flce_set_schedule({"recompute": flce.FLCE_SCHEDULE_RECOMPUTE,
-                                   "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD,
-                                   "fused_fwd_dw_once": flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE}
-                                  [sched])
+                                   "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD}[sched])
     try:
         ref = flce.fused(X, W, lab, softcap=cap, dloss=0.5, dw_fp32=dw_fp32)
         events = [torch.cuda.Event() for _ in range(n_slices)]
@@ -135,11 +132,9 @@ def test_sliced_dW_equals_unsliced(sched, n_slices, dw_fp32, cuda_device):
     bounds = flce.dw_slice_bounds(V, n_slices)
     assert bounds[0][0] == 0 and bounds[-1][1] == V
     assert all(b0 == a1 for (_, b0), (a1, _) in zip(bounds, bounds[1:]))
-    nonempty = sum(b > a for a, b in bounds)
-    if sched == "fused_fwd":  # one dW GEMM per row chunk at this shape
+    if sched == "fused_fwd":
+        nonempty = sum(b > a for a, b in bounds)
         assert names.count("dw_acc_gemm") == names.count("lse_q_gemm") - 1 + nonempty
-    if sched == "fused_fwd_dw_once":
-        assert names.count("lse_q_gemm") == 2 and names.count("dw_acc_gemm") == nonempty
 
 
 def test_fused_dp_sliced_and_sharded_one_rank_nccl(cuda_device):

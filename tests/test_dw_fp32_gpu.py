@@ -17,8 +17,7 @@ from parity import TOL, rel_fro, rel_scalar, run_oracle, to_np
 pytestmark = pytest.mark.gpu
 
 SCHEDULES = {"recompute": flce.FLCE_SCHEDULE_RECOMPUTE,
-             "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD,
-             "fused_fwd_dw_once": flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE}
+             "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD}
 
 
 class _schedule:

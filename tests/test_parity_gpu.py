@@ -49,8 +49,7 @@ class schedule:
 
 
 SCHEDULES = {"recompute": flce.FLCE_SCHEDULE_RECOMPUTE,
-             "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD,
-             "fused_fwd_dw_once": flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE}
+             "fused_fwd": flce.FLCE_SCHEDULE_FUSED_FORWARD}
 
 
 def _inputs(BT, H, V, dtype, ignore_frac, seed, device):
@@ -63,7 +62,7 @@ def _inputs(BT, H, V, dtype, ignore_frac, seed, device):
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "%dx%dx%d-%s-cap%g" % c[:5])
 def test_fused_matches_oracle(case, sched, cuda_device):
     BT, H, V, dtype, softcap, ign, seed = case
-    if dtype == "fp32" and sched.startswith("fused_fwd"):
+    if dtype == "fp32" and sched == "fused_fwd":
         pytest.skip("fp32 problems always use the recompute schedule")
     X, W, lab, Xd, Wd, labd = _inputs(BT, H, V, dtype, ign, seed, cuda_device)
     o = run_oracle(X, W, lab, softcap=softcap, dloss=0.5)
@@ -170,28 +169,22 @@ def test_launch_count_and_stream(cuda_device):
     s.synchronize()
     ref = flce.fused(Xd, Wd, labd)
     assert torch.equal(ref[1], dX)
+    with schedule(flce.FLCE_SCHEDULE_FUSED_FORWARD):
+        flce.flce_profile_start(64)
+        flce.fused(Xd, Wd, labd)
+        n = flce.flce_last_launch_count()
+        names = [k for k, _ in flce.flce_profile_stop()]
     # labels, 2 row chunks x (forward GEMM, lse_q, recomputation GEMM (returns
-    # at once: nothing flagged), lse_q, dX GEMM [+ split reduce], then the
-    # chunk's dW GEMM, or one dW GEMM over both chunks after the last), finalize
+    # at once: nothing flagged), lse_q, dX GEMM [+ split reduce], dW GEMM),
+    # finalize
+    assert len(names) == n
     chunk = ["lse_q_gemm", "lse_q", "lse_q_repair_gemm", "lse_q", "dx_gemm"]
-    for which, once in ((flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK, False),
-                        (flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE, True),
-                        # the rule at this shape: 256 x 2048 q (1 MiB) is no more than
-                        # a chunk's q (0.5 MiB) plus the fp32 sum (1 MB)
-                        (flce.FLCE_SCHEDULE_FUSED_FORWARD, True)):
-        with schedule(which):
-            flce.flce_profile_start(64)
-            flce.fused(Xd, Wd, labd)
-            n = flce.flce_last_launch_count()
-            names = [k for k, _ in flce.flce_profile_stop()]
-        assert len(names) == n
-        body = names[1:-1]
-        red = ["dx_reduce"] if "dx_reduce" in body else []
-        assert names[0] == "labels" and names[-1] == "loss_finalize"
-        if once:
-            assert body == (chunk + red) * 2 + ["dw_acc_gemm"]
-        else:
-            assert body == (chunk + red + ["dw_acc_gemm"]) * 2
+    tail = ["dw_acc_gemm"]
+    body = names[1:-1]
+    if "dx_reduce" in body:
+        tail = ["dx_reduce"] + tail
+    assert names[0] == "labels" and names[-1] == "loss_finalize"
+    assert body == (chunk + tail) * 2
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(cuda_device):
@@ -348,86 +341,3 @@ def test_rows_outside_the_shared_reference_range(cap, H, cuda_device):
         nrm = np.linalg.norm(ref)
         got = to_np(dX[i:i + 1])[0]
         assert (nrm == 0 and not got.any()) or np.linalg.norm(got - ref) <= 2e-2 * nrm, i
-
-
-def _ws_fused(BT, H, V, which):
-    with schedule(which):
-        return flce.flce_workspace_size(flce.make_problem(BT, H, V), flce.FLCE_OP_FUSED)
-
-
-@pytest.mark.parametrize("case", [(1100, 512, 3000, 0.0, 0.05, 41),
-                                  (1300, 256, 4100, 10.0, 0.10, 42)],
-                         ids=lambda c: "%dx%dx%d-cap%g" % c[:4])
-def test_dw_once_and_per_chunk_match_oracle(case, cuda_device):
-    """Fused-in-forward schedule on two row chunks (the last ragged): dW as
-    one GEMM over every row and as one GEMM per chunk summed in fp32 both
-    match the oracle; the forward and dX GEMMs run the same chunks either
-    way, so loss and dX are bitwise equal, and the two dW differ only by the
-    order of the fp32 sums before the one bf16 rounding.  The automatic
-    choice follows the memory rule: every row's q held when it takes no
-    more than one chunk's q plus the fp32 V x H sum."""
-    BT, H, V, cap, ign, seed = case
-    X, W, lab, Xd, Wd, labd = _inputs(BT, H, V, "bf16", ign, seed, cuda_device)
-    o = run_oracle(X, W, lab, softcap=cap, dloss=0.5)
-    out = {}
-    for name, which in (("fused_fwd_dw_once", flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE),
-                        ("fused_fwd_dw_per_chunk", flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK)):
-        with schedule(which):
-            flce.flce_profile_start(64)
-            out[name] = flce.fused(Xd, Wd, labd, softcap=cap, dloss=0.5)
-            kinds = [k for k, _ in flce.flce_profile_stop()]
-        assert kinds.count("lse_q_gemm") == 2
-        assert kinds.count("dw_acc_gemm") == (1 if name.endswith("once") else 2)
-        loss, dX, dW = out[name]
-        tol = TOL["bf16"]
-        assert rel_scalar(loss.item(), o["loss"]) <= tol["loss"], (name, loss.item(), o["loss"])
-        assert rel_fro(to_np(dX), o["dX"]) <= tol["grad"], name
-        assert rel_fro(to_np(dW), o["dW"]) <= tol["grad"], name
-    a, b = out["fused_fwd_dw_once"], out["fused_fwd_dw_per_chunk"]
-    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
-    assert rel_fro(to_np(a[2]), to_np(b[2]).astype(np.float64)) <= 2e-3
-    ldp = -(-V // 256) * 256
-    cb = -(-(-(-BT // 2)) // 128) * 128
-    once_by_rule = BT * ldp * 2 <= cb * ldp * 2 + V * H * 4
-    auto = _ws_fused(BT, H, V, flce.FLCE_SCHEDULE_AUTO)
-    once = _ws_fused(BT, H, V, flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE)
-    per_chunk = _ws_fused(BT, H, V, flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK)
-    assert auto == (once if once_by_rule else per_chunk) and once != per_chunk
-    assert once_by_rule == (H == 512)
-
-
-def test_dw_once_three_chunks_matches_per_chunk(cuda_device):
-    """Three row chunks (1024, 1024 and a ragged 852 rows: H = 16384 keeps a
-    chunk's X rows within 46 MiB): one dW GEMM over all 2900 rows against
-    three summed in fp32, with the fp32 dW too; loss and dX bitwise equal,
-    dW equal up to the order of the fp32 sums.  The one dW GEMM's Xs (95 MB)
-    exceeds what stays in L2, so its waves of tiles alternate their K
-    direction; a tile's direction follows its place in the whole dW, so the
-    same GEMM in vocabulary slices gives the same bits."""
-    BT, H, V = 2900, 16384, 500
-    X, W, lab = inputs.make_inputs(BT, H, V, "bf16", 1.0, 0.02, 0.05, 43, device=cuda_device)
-    res = {}
-    for name, which in (("once", flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE),
-                        ("per_chunk", flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_PER_CHUNK)):
-        for dw32 in (False, True):
-            with schedule(which):
-                flce.flce_profile_start(64)
-                res[name, dw32] = flce.fused(X, W, lab, softcap=5.0, dloss=0.5, dw_fp32=dw32)
-                kinds = [k for k, _ in flce.flce_profile_stop()]
-            assert kinds.count("lse_q_gemm") == 3
-            assert kinds.count("dw_acc_gemm") == (1 if name == "once" else 3)
-    torch.cuda.synchronize()
-    for dw32 in (False, True):
-        a, b = res["once", dw32], res["per_chunk", dw32]
-        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
-        assert torch.isfinite(a[2]).all()
-        da, db = a[2].double(), b[2].double()
-        assert float((da - db).norm() / db.norm()) <= (2e-3 if not dw32 else 1e-5)
-    # the bf16 dW is the rounding of the fp32 one
-    assert torch.equal(res["once", True][2].to(torch.bfloat16), res["once", False][2])
-    events = [torch.cuda.Event() for _ in range(2)]
-    with schedule(flce.FLCE_SCHEDULE_FUSED_FORWARD_DW_ONCE):
-        sliced = flce.fused(X, W, lab, softcap=5.0, dloss=0.5, slice_events=events)
-    torch.cuda.synchronize()
-    for a, b in zip(sliced, res["once", False]):
-        assert torch.equal(a, b)
